@@ -1,0 +1,177 @@
+/*
+ * lq.h -- C ABI of the B200 (sm_100a) LiquidQuant W4A8 GEMM library.
+ *
+ * The method: "LiquidGEMM: Hardware-Efficient W4A8 GEMM Kernel for
+ * High-Performance LLM Serving" (arXiv 2509.01229), as described on its
+ * pith.science review page.  Weights go through two levels of quantization
+ * (LiquidQuant, "LQQ"): per-channel symmetric INT8 in the protective range
+ * [-119, 119], then group-wise UINT4 with an integer UINT8 scale s_u8 and an
+ * offset a = 2^7 + min(Q_i8) per group of 64 along K.  Inside the GEMM each
+ * 4-bit code is expanded back to INT8 with the overflow-free identity
+ * Q_i8_hat = (Q_u4 * s_u8 + a) XOR 0x80, and the INT8 x INT8 product is
+ * accumulated in int32 on the tensor cores.
+ *
+ * Conventions for every entry point
+ *   - All pointers are DEVICE pointers unless stated otherwise.  The caller
+ *     owns every buffer; the library never allocates or frees device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  All work is enqueued asynchronously on it; nothing blocks the
+ *     host except lq_get_device_error.
+ *   - Arguments are validated before anything is launched; on any error
+ *     nothing is launched and nothing is written.
+ *   - Matrices are row-major.  Activations X and x_q are [M, K] (M tokens),
+ *     weights W are [N, K] (nn.Linear layout, N output features), the output
+ *     is [M, N].  bf16 buffers are passed as void*.
+ *   - Only compute capability 10.0 devices (B200, sm_100a) are supported.
+ *   - Inputs must be finite; non-finite values give unspecified codes but no
+ *     fault.
+ *
+ * Packed weight format (this library's own; the paper's "dual-MMA packed
+ * layout" is not given on the page):
+ *   qw   uint8 [N, K/2]: in row n, little-endian 32-bit word j holds codes
+ *        k = 8j..8j+7, byte b (0..3) = code[8j+b] | code[8j+4+b] << 4, so one
+ *        AND yields codes 8j..8j+3 and one shift + AND yields 8j+4..8j+7,
+ *        each already in byte order for a 4-wide SWAR expansion.
+ *   s_u8 uint8 [K/64, N] and a_u8 uint8 [K/64, N]: per-group scale and
+ *        offset, N contiguous.
+ *   s_c  float [N]: per-channel scale of level 1 (amax / 119).
+ */
+#ifndef LQ_H
+#define LQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LQ_API __attribute__((visibility("default")))
+#else
+#define LQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lq_status {
+  LQ_OK = 0,
+  LQ_ERR_INVALID_ARG = 1,       /* NULL pointer where data is needed, negative size */
+  LQ_ERR_UNSUPPORTED_SHAPE = 2, /* a size rule below is broken */
+  LQ_ERR_MISALIGNED = 3,        /* a pointer is not aligned as required */
+  LQ_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
+  LQ_ERR_CUDA = 5,              /* a CUDA runtime or driver call failed */
+  LQ_ERR_TIMEOUT = 6,           /* a device-side bounded wait gave up (reported by
+                                   lq_get_device_error) */
+  LQ_ERR_ARCH = 7               /* the current device is not compute capability 10.0 */
+} lq_status;
+
+/* Group size along K of the level-2 quantization (the paper's default). */
+#define LQ_GROUP 64
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+LQ_API int lq_version(void);
+
+/* Human-readable name of a status code (static storage). */
+LQ_API const char* lq_status_string(lq_status status);
+
+/*
+ * lq_quantize_weights -- offline LiquidQuant of a weight matrix (both levels).
+ *   Level 1 (review page: referee summary and circularity rationale, the
+ *   protective range "Q_i8 in [-119,119]"):
+ *     amax_n = max_k |W[n,k]|;  Q_i8 = clamp(rint(W * (119 / amax_n)), -119, 119)
+ *     s_c[n] = amax_n / 119;    a zero row gets s_c = 1 and codes 0.
+ *   Level 2 (review page: referee summary; major comment 3 and minor comment 2
+ *   on the integer scale; "What carries the argument" for the offset):
+ *     per group of 64 along K: mn = min Q_i8, R = max Q_i8 - mn,
+ *     s_u8 = max(1, round(R / 15)), a = 128 + mn,
+ *     Q_u4 = min(15, round_half_up((Q_i8 - mn) / s_u8)).
+ *   Rounding: float ops are single IEEE binary32 operations; rint is round to
+ *   nearest even.
+ *   W_bf16  [N, K] bf16, 16-byte aligned.
+ *   qw      [N, K/2] uint8 out, 16-byte aligned.
+ *   s_u8, a_u8 [K/64, N] uint8 out.   s_c [N] float out.
+ *   group must be 64.  Requires N >= 1, K >= 64, K % 64 == 0.
+ */
+LQ_API lq_status lq_quantize_weights(const void* W_bf16, int N, int K, int group, uint8_t* qw,
+                              uint8_t* s_u8, uint8_t* a_u8, float* s_c, void* stream);
+
+/*
+ * lq_quantize_act -- per-token symmetric INT8 activations (the review page's
+ * "8-bit activations"; symmetric per token in [-127, 127] is this library's
+ * reading):
+ *   amax_m = max_k |X[m,k]|;  x_q = clamp(rint(X * (127 / amax_m)), -127, 127)
+ *   s_x[m] = amax_m / 127;    a zero row gets s_x = 1 and codes 0.
+ *   X_bf16 [M, K] bf16 and x_q [M, K] int8 out, both 16-byte aligned.
+ *   s_x [M] float out.  Requires K % 16 == 0; M == 0 is a no-op.
+ */
+LQ_API lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, float* s_x, void* stream);
+
+/*
+ * lq_w4a8_gemm -- the W4A8 GEMM (review page: the abstract and referee
+ * summary; the loop nest of Figure 2):
+ *   W_hat[n,k] = int8((Q_u4[n,k] * s_u8[g,n] + a_u8[g,n]) XOR 0x80),  g = k / 64
+ *   acc[m,n]   = sum_k x_q[m,k] * W_hat[n,k]          (exact, int32)
+ *   out[m,n]   = bf16_rne(float(acc) * (s_x[m] * s_c[n]))
+ *   x_q [M, K] int8, qw [N, K/2], s_u8/a_u8 [K/64, N] uint8: 16-byte aligned.
+ *   s_x [M], s_c [N] float: 4-byte aligned.  out_bf16 [M, N] bf16 out.
+ *   Requires group == 64, K % 128 == 0, 128 <= K <= 131072, N % 16 == 0,
+ *   N >= 16; M == 0 is a no-op.
+ *   workspace: device scratch of at least lq_w4a8_gemm_workspace_size(M,N,K)
+ *   bytes (may be NULL when that is 0), 16-byte aligned, ZERO-FILLED by the
+ *   caller before its first use.  Each call leaves it zero-filled again, so
+ *   it can be reused by later calls on the same stream without clearing; two
+ *   calls in flight at the same time must not share one.  After a call that
+ *   ended in LQ_ERR_TIMEOUT the caller must clear it again.
+ */
+LQ_API size_t lq_w4a8_gemm_workspace_size(int M, int N, int K);
+LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                       const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c,
+                       void* out_bf16, int M, int N, int K, int group, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * lq_w4a8_gemm_ex -- lq_w4a8_gemm with the schedule chosen by the caller
+ * (tests and tuning).  block_t: tokens per tile, one of 16, 32, 64, 128, 256,
+ * or 0 for the automatic choice.  grid: number of CTAs, 0 for automatic; the
+ * M x N x K work is cut into K-blocks of 128 and spread evenly over the CTAs
+ * (stream-K), and tiles shared by several CTAs are reduced through the
+ * workspace.  grid is clamped to the number of K-blocks of work.
+ * out_i32: when nonzero, out receives the int32 accumulators acc[m,n]
+ * instead of bf16 (bit-exact check of the contraction).
+ */
+LQ_API size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int grid);
+LQ_API lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                          const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c, void* out,
+                          int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
+                          int block_t, int grid, int out_i32, void* stream);
+
+/*
+ * lq_w4a8_gemm_i32 -- the contraction only: acc[m,n] as int32 [M, N] (16-byte
+ * aligned), same operands, rules and workspace as lq_w4a8_gemm.
+ */
+LQ_API lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* s_u8,
+                           const uint8_t* a_u8, int32_t* acc, int M, int N, int K, int group,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * lq_dequant_weights_i8 -- the in-kernel LiquidQuant expansion written out
+ * (review page: "What carries the argument"; Eq. 12 in the circularity
+ * rationale): w_i8[n,k] = int8((Q_u4 * s_u8 + a) XOR 0x80), [N, K] int8 out,
+ * 16-byte aligned.  Uses the same device routine as the GEMM.  Requires
+ * group == 64, K % 64 == 0, N >= 1.
+ */
+LQ_API lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8, int N,
+                                int K, int group, int8_t* w_i8, void* stream);
+
+/*
+ * lq_get_device_error -- synchronizes `stream`, then reads and clears the
+ * library's device error word.  Returns LQ_ERR_TIMEOUT if a kernel gave up a
+ * bounded wait since the last call (its output is then undefined),
+ * LQ_ERR_CUDA if the synchronization itself failed, else LQ_OK.
+ */
+LQ_API lq_status lq_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LQ_H */

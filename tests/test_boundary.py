@@ -1,0 +1,85 @@
+"""The C ABI on the CPU: the library loads, exports every entry point declared in
+include/lq.h, and rejects bad arguments before touching a device (no GPU needed)."""
+import ctypes
+
+import pytest
+
+import w4a8_bit_weight_b200 as lq
+from w4a8_bit_weight_b200 import build as lqbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lqbuild.build()
+    return lq.load_library()
+
+
+def test_exports_every_header_symbol(lib):
+    names = lq.header_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert "lq_quantize_weights" in names and "lq_quantize_act" in names and "lq_w4a8_gemm" in names
+
+
+def test_version_and_status_strings(lib):
+    assert lq.lq_version() >= 100
+    for code in range(8):
+        s = lq.lq_status_string(code)
+        assert s.startswith(lq.STATUS[code])
+
+
+P = ctypes.c_void_p
+GOOD = P(1 << 20)      # a 16-byte aligned fake address; never dereferenced on these paths
+ODD = P((1 << 20) + 8)
+
+
+def gemm(lib, M=16, N=256, K=512, group=64, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=GOOD, sc=GOOD, out=GOOD,
+         bt=0, grid=0):
+    return lib.lq_w4a8_gemm_ex(x, sx, qw, s, a, sc, out, M, N, K, group, None, 0, bt, grid, 0, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(group=32), 2), (dict(K=192), 2), (dict(K=64), 2), (dict(K=0), 2), (dict(K=262144), 2),
+    (dict(N=8), 2), (dict(N=200), 2), (dict(N=0), 2),
+    (dict(M=-1), 1), (dict(N=-16), 1),
+    (dict(x=P(0)), 1), (dict(qw=P(0)), 1), (dict(s=P(0)), 1), (dict(a=P(0)), 1), (dict(out=P(0)), 1),
+    (dict(sx=P(0)), 1), (dict(sc=P(0)), 1),
+    (dict(x=ODD), 3), (dict(qw=ODD), 3), (dict(s=ODD), 3), (dict(a=ODD), 3), (dict(out=ODD), 3),
+    (dict(sx=P((1 << 20) + 2)), 3),
+    (dict(bt=48), 1), (dict(grid=-1), 1),
+])
+def test_gemm_rejects_before_launch(lib, kw, code):
+    assert gemm(lib, **kw) == code
+
+
+def test_gemm_empty_batch_is_a_noop(lib):
+    # M == 0: nothing to do and no device touched, even with NULL buffers
+    assert lib.lq_w4a8_gemm(None, None, None, None, None, None, None, 0, 256, 512, 64, None, 0, None) == 0
+
+
+def test_quantize_rejects_before_launch(lib):
+    q = lib.lq_quantize_weights
+    assert q(GOOD, 16, 96, 64, GOOD, GOOD, GOOD, GOOD, None) == 2      # K % 64
+    assert q(GOOD, 16, 128, 32, GOOD, GOOD, GOOD, GOOD, None) == 2     # group
+    assert q(GOOD, 0, 128, 64, GOOD, GOOD, GOOD, GOOD, None) == 2      # N >= 1
+    assert q(None, 16, 128, 64, GOOD, GOOD, GOOD, GOOD, None) == 1
+    assert q(ODD, 16, 128, 64, GOOD, GOOD, GOOD, GOOD, None) == 3
+    a = lib.lq_quantize_act
+    assert a(GOOD, 4, 24, GOOD, GOOD, None) == 2                        # K % 16
+    assert a(GOOD, -1, 64, GOOD, GOOD, None) == 1
+    assert a(None, 0, 64, None, None, None) == 0                        # empty batch
+    assert a(ODD, 4, 64, GOOD, GOOD, None) == 3
+    d = lib.lq_dequant_weights_i8
+    assert d(GOOD, GOOD, GOOD, 16, 100, 64, GOOD, None) == 2
+    assert d(GOOD, GOOD, GOOD, 16, 128, 64, ODD, None) == 3
+
+
+def test_workspace_size_rules(lib):
+    # invalid shapes need no workspace; the query never touches a device
+    assert lib.lq_w4a8_gemm_workspace_size(16, 200, 512) == 0
+    assert lib.lq_w4a8_gemm_workspace_size(0, 256, 512) == 0
+    # one CTA per tile (grid = tiles): no tile is shared, no workspace
+    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 2) == 0
+    # 3 CTAs over 2 tiles x 4 K-blocks: split tiles need [tiles][16][128] int32 + tickets
+    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 3) == 2 * 16 * 128 * 4 + 16

@@ -1,1 +1,247 @@
-"""placeholder"""
+"""B200 (sm_100a) LiquidQuant W4A8 GEMM -- Python binding of the C ABI in include/lq.h.
+
+Argument marshalling only: every step of the path runs in the CUDA library
+``liblq_b200.so`` built in-tree (``python -m w4a8_bit_weight_b200.build``).
+PyTorch supplies device memory and the current stream.  There is no CPU
+fallback: calling any op without the built library, or on a device that is
+not compute capability 10.0, raises.
+
+Functions keep the C names:
+    lq_quantize_weights(W)                       -> (qw, s_u8, a_u8, s_c)
+    lq_quantize_act(X)                           -> (x_q, s_x)
+    lq_w4a8_gemm(x_q, s_x, qw, s_u8, a_u8, s_c)  -> out bf16 [M, N]
+    lq_w4a8_gemm_i32(x_q, qw, s_u8, a_u8)        -> acc int32 [M, N]
+    lq_dequant_weights_i8(qw, s_u8, a_u8)        -> w_i8 int8 [N, K]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblq_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lq.h")
+GROUP = 64
+
+STATUS = {
+    0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED_SHAPE", 3: "LQ_ERR_MISALIGNED",
+    4: "LQ_ERR_WORKSPACE", 5: "LQ_ERR_CUDA", 6: "LQ_ERR_TIMEOUT", 7: "LQ_ERR_ARCH",
+}
+
+
+class LQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {STATUS.get(status, status)}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library not built: {path} is missing "
+                               "(run python -m w4a8_bit_weight_b200.build)")
+        lib = ctypes.CDLL(path)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        sig = {
+            "lq_version": ([], I),
+            "lq_status_string": ([I], ctypes.c_char_p),
+            "lq_quantize_weights": ([P, I, I, I, P, P, P, P, P], I),
+            "lq_quantize_act": ([P, I, I, P, P, P], I),
+            "lq_w4a8_gemm_workspace_size": ([I, I, I], Z),
+            "lq_w4a8_gemm_workspace_size_ex": ([I, I, I, I, I], Z),
+            "lq_w4a8_gemm": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, P], I),
+            "lq_w4a8_gemm_ex": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, I, I, I, P], I),
+            "lq_w4a8_gemm_i32": ([P, P, P, P, P, I, I, I, I, P, Z, P], I),
+            "lq_dequant_weights_i8": ([P, P, P, I, I, I, P, P], I),
+            "lq_get_device_error": ([P], I),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+def header_symbols(path: str = HEADER_PATH):
+    """Names of the entry points declared in include/lq.h."""
+    with open(path) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^LQ_API\s+[\w\s\*]+?\b(lq_\w+)\s*\(", text, re.M)))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise LQError(fn, st)
+
+
+def _need(t: torch.Tensor, dtype, name: str, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+# ----------------------------------------------------------------------------
+# workspace: one zero-filled scratch buffer per device, grown on demand.  The
+# kernels leave it zero-filled after every call, so it is cleared only once.
+# ----------------------------------------------------------------------------
+_ws = {}
+
+
+def workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    buf = _ws.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
+        _ws[key] = buf
+    return buf
+
+
+def lq_version() -> int:
+    return load_library().lq_version()
+
+
+def lq_status_string(status: int) -> str:
+    return load_library().lq_status_string(status).decode()
+
+
+def lq_quantize_weights(W: torch.Tensor, group: int = GROUP, out=None):
+    """Offline LiquidQuant of W [N, K] bf16 -> (qw [N,K/2] u8, s_u8 [K/64,N] u8, a_u8 [K/64,N] u8, s_c [N] f32)."""
+    lib = load_library()
+    _need(W, torch.bfloat16, "W")
+    N, K = W.shape
+    dev = W.device
+    if out is None:
+        out = (torch.empty(N, K // 2, dtype=torch.uint8, device=dev),
+               torch.empty(max(K // group, 0), N, dtype=torch.uint8, device=dev),
+               torch.empty(max(K // group, 0), N, dtype=torch.uint8, device=dev),
+               torch.empty(N, dtype=torch.float32, device=dev))
+    qw, s, a, sc = out
+    with torch.cuda.device(dev):
+        _check("lq_quantize_weights", lib.lq_quantize_weights(
+            _ptr(W), N, K, group, _ptr(qw), _ptr(s), _ptr(a), _ptr(sc), _stream(dev)))
+    return qw, s, a, sc
+
+
+def lq_quantize_act(X: torch.Tensor, out=None):
+    """Per-token symmetric INT8 of X [M, K] bf16 -> (x_q [M,K] int8, s_x [M] f32)."""
+    lib = load_library()
+    _need(X, torch.bfloat16, "X")
+    M, K = X.shape
+    if out is None:
+        out = (torch.empty(M, K, dtype=torch.int8, device=X.device),
+               torch.empty(M, dtype=torch.float32, device=X.device))
+    xq, sx = out
+    with torch.cuda.device(X.device):
+        _check("lq_quantize_act", lib.lq_quantize_act(_ptr(X), M, K, _ptr(xq), _ptr(sx), _stream(X.device)))
+    return xq, sx
+
+
+def lq_w4a8_gemm_workspace_size(M: int, N: int, K: int, block_t: int = 0, grid: int = 0) -> int:
+    lib = load_library()
+    if block_t == 0 and grid == 0:
+        return int(lib.lq_w4a8_gemm_workspace_size(M, N, K))
+    return int(lib.lq_w4a8_gemm_workspace_size_ex(M, N, K, block_t, grid))
+
+
+def _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, grid, out_i32, ws):
+    lib = load_library()
+    _need(x_q, torch.int8, "x_q")
+    M, K = x_q.shape
+    N = qw.shape[0]
+    _need(qw, torch.uint8, "qw", (N, K // 2))
+    _need(s_u8, torch.uint8, "s_u8", (K // group, N))
+    _need(a_u8, torch.uint8, "a_u8", (K // group, N))
+    if not out_i32:
+        _need(s_x, torch.float32, "s_x", (M,))
+        _need(s_c, torch.float32, "s_c", (N,))
+    odt = torch.int32 if out_i32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(M, N, dtype=odt, device=x_q.device)
+    _need(out, odt, "out", (M, N))
+    with torch.cuda.device(x_q.device):
+        need = lq_w4a8_gemm_workspace_size(M, N, K, block_t, grid)
+        if ws is None:
+            ws = workspace(need, x_q.device)
+        nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+        _check("lq_w4a8_gemm", lib.lq_w4a8_gemm_ex(
+            _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out),
+            M, N, K, group, _ptr(ws), nbytes, block_t, grid, 1 if out_i32 else 0, _stream(x_q.device)))
+    return out
+
+
+def lq_w4a8_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP,
+                 block_t: int = 0, grid: int = 0, workspace_buf=None):
+    """W4A8 GEMM: bf16(float(x_q @ dequant(qw)^T) * s_x[m] * s_c[n]) -> [M, N] bf16."""
+    return _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, grid, False, workspace_buf)
+
+
+def lq_w4a8_gemm_i32(x_q, qw, s_u8, a_u8, out=None, group: int = GROUP, block_t: int = 0,
+                     grid: int = 0, workspace_buf=None):
+    """The int32 accumulators x_q @ dequant(qw)^T -> [M, N] int32."""
+    return _gemm(x_q, None, qw, s_u8, a_u8, None, out, group, block_t, grid, True, workspace_buf)
+
+
+def lq_dequant_weights_i8(qw, s_u8, a_u8, group: int = GROUP, out=None):
+    """LiquidQuant expansion written out: int8((q*s + a) XOR 0x80) -> [N, K] int8."""
+    lib = load_library()
+    N, K = qw.shape[0], qw.shape[1] * 2
+    _need(qw, torch.uint8, "qw")
+    _need(s_u8, torch.uint8, "s_u8", (K // group, N))
+    _need(a_u8, torch.uint8, "a_u8", (K // group, N))
+    if out is None:
+        out = torch.empty(N, K, dtype=torch.int8, device=qw.device)
+    with torch.cuda.device(qw.device):
+        _check("lq_dequant_weights_i8", lib.lq_dequant_weights_i8(
+            _ptr(qw), _ptr(s_u8), _ptr(a_u8), N, K, group, _ptr(out), _stream(qw.device)))
+    return out
+
+
+def lq_get_device_error(device=None) -> int:
+    """Synchronizes the current stream; returns and clears the library's device error status."""
+    lib = load_library()
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        return int(lib.lq_get_device_error(_stream(dev)))
+
+
+class W4A8Linear:
+    """A linear layer y = x W^T with LiquidQuant W4A8 weights, quantized once at construction."""
+
+    def __init__(self, weight: torch.Tensor):
+        self.N, self.K = weight.shape
+        self.qw, self.s_u8, self.a_u8, self.s_c = lq_quantize_weights(weight.contiguous())
+
+    def __call__(self, x: torch.Tensor) -> torch.Tensor:
+        x_q, s_x = lq_quantize_act(x.contiguous())
+        return lq_w4a8_gemm(x_q, s_x, self.qw, self.s_u8, self.a_u8, self.s_c)

@@ -1,0 +1,333 @@
+// lq_api.cu -- the C ABI (include/lq.h): argument validation, schedule choice,
+// TMA descriptors and kernel launches.  All device code of the library is in
+// this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/lq.h"
+#include "lq_device.cuh"
+#include "lq_gemm_kernel.cuh"
+#include "lq_quant_kernels.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool sm100 = false;
+  int sms = 0;
+  bool attr_set[16] = {};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+lq_status current_device(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LQ_ERR_CUDA;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d.ready) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LQ_ERR_CUDA;
+      d.sm100 = (major == 10 && minor == 0);
+      d.sms = sms;
+      d.ready = true;
+    }
+  }
+  *out = &d;
+  return d.sm100 ? LQ_OK : LQ_ERR_ARCH;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D byte-element tensor [outer][inner] with `row_bytes` between rows.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- schedule
+struct Schedule {
+  int bt = 0;        // tokens per tile
+  int tiles_m = 0, tiles_n = 0, KB = 0;
+  long long tiles = 0, U = 0;
+  int grid = 0;
+  bool split = false;  // some tile is shared by several CTAs
+  size_t ws_bytes = 0;
+};
+
+int auto_block_t(int M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  return 128;
+}
+
+bool valid_block_t(int bt) { return bt == 16 || bt == 32 || bt == 64 || bt == 128 || bt == 256; }
+
+Schedule make_schedule(int M, int N, int K, int block_t, int grid, int sms) {
+  Schedule s;
+  s.bt = block_t ? block_t : auto_block_t(M);
+  s.tiles_m = (M + s.bt - 1) / s.bt;
+  s.tiles_n = (N + lq::kBlockN - 1) / lq::kBlockN;
+  s.KB = K / lq::kBlockK;
+  s.tiles = (long long)s.tiles_m * s.tiles_n;
+  s.U = s.tiles * s.KB;
+  long long g = grid;
+  if (g <= 0) {
+    // enough whole tiles for two waves: one CTA per tile; else spread K-blocks
+    // evenly over one CTA per SM (stream-K)
+    g = (s.tiles >= 2LL * sms) ? s.tiles : (long long)sms;
+  }
+  if (g > s.U) g = s.U;
+  if (g > INT_MAX) g = INT_MAX;
+  if (g < 1) g = 1;
+  s.grid = (int)g;
+  s.split = false;
+  for (long long c = 1; c < g; ++c)
+    if ((c * s.U / g) % s.KB != 0) {
+      s.split = true;
+      break;
+    }
+  if (s.split) {
+    const size_t acc = (size_t)s.tiles * s.bt * lq::kBlockN * sizeof(int32_t);
+    s.ws_bytes = acc + (((size_t)s.tiles * sizeof(unsigned) + 15) / 16) * 16;
+  }
+  return s;
+}
+
+lq_status check_gemm_shape(int M, int N, int K, int group) {
+  if (M < 0 || N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (group != LQ_GROUP) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (K < lq::kBlockK || K % lq::kBlockK != 0 || K > 131072) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (N < 16 || N % 16 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return LQ_OK;
+}
+
+template <int BT, bool I32>
+lq_status launch_gemm_t(const Schedule& s, DeviceInfo* dev, const CUtensorMap& tx, const CUtensorMap& tw,
+                        const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  using C = lq::GemmCfg<BT>;
+  auto kern = lq::w4a8_gemm_kernel<BT, I32>;
+  const int slot = (BT == 16 ? 0 : BT == 32 ? 1 : BT == 64 ? 2 : BT == 128 ? 3 : 4) + (I32 ? 5 : 0);
+  if (!dev->attr_set[slot]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return LQ_ERR_CUDA;
+    dev->attr_set[slot] = true;
+  }
+  kern<<<s.grid, lq::kGemmThreads, C::kSmemBytes, st>>>(tx, tw, ts, ta, a);
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+template <bool I32>
+lq_status launch_gemm(const Schedule& s, DeviceInfo* dev, const CUtensorMap& tx, const CUtensorMap& tw,
+                      const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  switch (s.bt) {
+    case 16: return launch_gemm_t<16, I32>(s, dev, tx, tw, ts, ta, a, st);
+    case 32: return launch_gemm_t<32, I32>(s, dev, tx, tw, ts, ta, a, st);
+    case 64: return launch_gemm_t<64, I32>(s, dev, tx, tw, ts, ta, a, st);
+    case 128: return launch_gemm_t<128, I32>(s, dev, tx, tw, ts, ta, a, st);
+    case 256: return launch_gemm_t<256, I32>(s, dev, tx, tw, ts, ta, a, st);
+  }
+  return LQ_ERR_INVALID_ARG;
+}
+
+lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                    const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
+                    void* workspace, size_t ws_bytes, int block_t, int grid, bool out_i32, void* stream) {
+  lq_status st = check_gemm_shape(M, N, K, group);
+  if (st != LQ_OK) return st;
+  if (block_t != 0 && !valid_block_t(block_t)) return LQ_ERR_INVALID_ARG;
+  if (grid < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0) return LQ_OK;
+  if (!x_q || !qw || !s_u8 || !a_u8 || !out || (!out_i32 && (!s_x || !s_c))) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x_q, 16) || !aligned(qw, 16) || !aligned(s_u8, 16) || !aligned(a_u8, 16) ||
+      !aligned(out, 16) || (s_x && !aligned(s_x, 4)) || (s_c && !aligned(s_c, 4)))
+    return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  const Schedule s = make_schedule(M, N, K, block_t, grid, dev->sms);
+  if (s.split) {
+    if (!workspace || ws_bytes < s.ws_bytes) return LQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return LQ_ERR_MISALIGNED;
+  }
+  CUtensorMap tx, tw, ts, ta;
+  if (!make_map_u8(&tx, x_q, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, s.bt,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, lq::kBlockK / 2, lq::kBlockN,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_u8(&ts, s_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, 2,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_u8(&ta, a_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, 2,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return LQ_ERR_CUDA;
+  lq::GemmArgs a;
+  a.s_x = s_x;
+  a.s_c = s_c;
+  a.out = out;
+  a.ws = s.split ? static_cast<int32_t*>(workspace) : nullptr;
+  a.ticket = s.split ? reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) +
+                                                        (size_t)s.tiles * s.bt * lq::kBlockN * 4)
+                     : nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = s.tiles_m;
+  a.KB = s.KB;
+  a.U = s.U;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return out_i32 ? launch_gemm<true>(s, dev, tx, tw, ts, ta, a, cs)
+                 : launch_gemm<false>(s, dev, tx, tw, ts, ta, a, cs);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lq_version(void) { return 100; }
+
+const char* lq_status_string(lq_status status) {
+  switch (status) {
+    case LQ_OK: return "LQ_OK";
+    case LQ_ERR_INVALID_ARG: return "LQ_ERR_INVALID_ARG: invalid argument";
+    case LQ_ERR_UNSUPPORTED_SHAPE: return "LQ_ERR_UNSUPPORTED_SHAPE: unsupported shape or group size";
+    case LQ_ERR_MISALIGNED: return "LQ_ERR_MISALIGNED: pointer not aligned as required";
+    case LQ_ERR_WORKSPACE: return "LQ_ERR_WORKSPACE: workspace missing or too small";
+    case LQ_ERR_CUDA: return "LQ_ERR_CUDA: a CUDA call failed";
+    case LQ_ERR_TIMEOUT: return "LQ_ERR_TIMEOUT: a device-side wait gave up";
+    case LQ_ERR_ARCH: return "LQ_ERR_ARCH: device is not compute capability 10.0";
+  }
+  return "unknown lq_status";
+}
+
+lq_status lq_quantize_weights(const void* W_bf16, int N, int K, int group, uint8_t* qw, uint8_t* s_u8,
+                              uint8_t* a_u8, float* s_c, void* stream) {
+  if (N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (group != LQ_GROUP || K < LQ_GROUP || K % LQ_GROUP != 0 || N < 1) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (!W_bf16 || !qw || !s_u8 || !a_u8 || !s_c) return LQ_ERR_INVALID_ARG;
+  if (!aligned(W_bf16, 16) || !aligned(qw, 16) || !aligned(s_c, 4)) return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  lq::quantize_weights_kernel<<<N, lq::kQuantWThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W_bf16), N, K, qw, s_u8, a_u8, s_c);
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, float* s_x, void* stream) {
+  if (M < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (K < 16 || K % 16 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return LQ_OK;
+  if (!X_bf16 || !x_q || !s_x) return LQ_ERR_INVALID_ARG;
+  if (!aligned(X_bf16, 16) || !aligned(x_q, 16) || !aligned(s_x, 4)) return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  lq::quantize_act_kernel<<<M, lq::kQuantActThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(X_bf16), K, x_q, s_x);
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int grid) {
+  if (check_gemm_shape(M, N, K, LQ_GROUP) != LQ_OK || M == 0) return 0;
+  if (block_t != 0 && !valid_block_t(block_t)) return 0;
+  DeviceInfo* dev = nullptr;
+  int sms = 148;
+  if (current_device(&dev) == LQ_OK) sms = dev->sms;
+  return make_schedule(M, N, K, block_t, grid, sms).ws_bytes;
+}
+
+size_t lq_w4a8_gemm_workspace_size(int M, int N, int K) {
+  return lq_w4a8_gemm_workspace_size_ex(M, N, K, 0, 0);
+}
+
+lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                          const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
+                          void* workspace, size_t workspace_bytes, int block_t, int grid, int out_i32,
+                          void* stream) {
+  return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out, M, N, K, group, workspace, workspace_bytes, block_t,
+                   grid, out_i32 != 0, stream);
+}
+
+lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                       const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K, int group,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes, 0, 0,
+                   false, stream);
+}
+
+lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8,
+                           int32_t* acc, int M, int N, int K, int group, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return gemm_impl(x_q, nullptr, qw, s_u8, a_u8, nullptr, acc, M, N, K, group, workspace, workspace_bytes, 0,
+                   0, true, stream);
+}
+
+lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8, int N, int K,
+                                int group, int8_t* w_i8, void* stream) {
+  if (N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (group != LQ_GROUP || K < LQ_GROUP || K % LQ_GROUP != 0 || N < 1) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (!qw || !s_u8 || !a_u8 || !w_i8) return LQ_ERR_INVALID_ARG;
+  if (!aligned(qw, 16) || !aligned(w_i8, 16)) return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  const long long words = (long long)N * (K / 8);
+  const int threads = 256;
+  const long long blocks = (words + threads - 1) / threads;
+  if (blocks > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
+  lq::dequant_weights_kernel<<<(int)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(qw), s_u8, a_u8, N, K, reinterpret_cast<uint32_t*>(w_i8));
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+lq_status lq_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LQ_ERR_CUDA;
+  unsigned int code = 0;
+  if (cudaMemcpyFromSymbol(&code, lq::g_error, sizeof code) != cudaSuccess) return LQ_ERR_CUDA;
+  if (code != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(lq::g_error, &zero, sizeof zero) != cudaSuccess) return LQ_ERR_CUDA;
+    return code == lq::kErrTimeout ? LQ_ERR_TIMEOUT : LQ_ERR_CUDA;
+  }
+  return LQ_OK;
+}
+
+}  // extern "C"
