@@ -1,0 +1,434 @@
+"""Benchmark of the B200 LiquidQuant W4A8 GEMM path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|mlp_up|tiny]
+    python bench.py --impl reference ...      # the CPU oracle on the host cores
+
+One step is one pass of the per-forward hot path over one batch: for every
+token count M of the workload, per-token INT8 quantization of the bf16
+activations followed by the W4A8 GEMM against a layer's packed weights (the
+weights are quantized offline, once, as in the method).  The default workload
+is the decode attention-projection layer, N = K = 4096, M in {1, 4, 16}.
+
+Timing: K steps are captured in one CUDA graph and replayed once between CUDA
+events on the launching stream, after W warm-up steps and about a second of
+untimed replays (so the clock sampler sees the GPU under load).  Each GEMM
+launch reads a different copy of the layer's packed weights, rotating over
+enough copies that the working set is several times the 126 MB L2, so every
+launch streams its weights from HBM.  External CUDA events around every GEMM
+node give the GEMM's own average duration for the roofline.
+
+With --gpus N > 1 (launched by torchrun) every rank runs an independent
+replica (the path has no exchange step); the time is the max over ranks and
+the value the sum of all ranks' work.
+
+Prints ONE JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 PFLOP/s int8 vs 2.25 bf16
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "mlp_up", "tiny"])
+    ap.add_argument("--soak-s", type=float, default=1.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# workload accounting
+# ---------------------------------------------------------------------------
+
+def gemm_bytes(M, N, K, G=64):
+    """Algorithmic HBM bytes of one GEMM: packed u4 weights, u8 scale and offset,
+    fp32 channel scales, int8 activations, fp32 token scales, bf16 output."""
+    return N * K // 2 + 2 * N * (K // G) + 4 * N + M * K + 4 * M + 2 * M * N
+
+
+def actq_bytes(M, K):
+    """bf16 activations in, int8 codes and fp32 scales out."""
+    return 2 * M * K + M * K + 4 * M
+
+
+def step_accounting(w):
+    gb = sum(gemm_bytes(M, w.N, w.K) for M in w.Ms)
+    ab = sum(actq_bytes(M, w.K) for M in w.Ms)
+    ops = sum(2 * M * w.N * w.K for M in w.Ms)
+    return gb, ab, ops
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "w4a8_bit_weight_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_gemm_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.proc = None
+        self.lines = []
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if gpu_uuid:
+            cmd += ["-i", gpu_uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.lines:
+            if ts < t0 or ts > t1:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU baseline: the oracle, as it stands, on the host cores
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(w, budget_s=10.0):
+    import oracle
+    from w4a8_bit_weight_b200 import synth
+    X, W = synth.make_workload(w)
+    o_qw, o_s, o_a, o_sc, _ = oracle.quantize_weights(synth.bf16_bits(W))
+    xb = synth.bf16_bits(X)
+    gb, ab, ops = step_accounting(w)
+    Ms = list(w.Ms)
+    # prefill-size layers: a bounded sample of token rows per step
+    rows = {M: min(M, 64) for M in Ms}
+    frac = sum(rows.values()) / sum(Ms)
+    t0 = time.perf_counter()
+    steps = 0
+    while True:
+        for M in Ms:
+            xq, sx = oracle.quantize_act(xb[:rows[M]])
+            oracle.w4a8_gemm(xq, sx, o_qw, o_s, o_a, o_sc)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    sample = (f"{steps} oracle steps, each quantize_act + w4a8_gemm (dequant, int64 contraction, "
+              f"epilogue) for M in {Ms}" + ("" if frac == 1 else f" with min(M,64) token rows") +
+              f", N={w.N}, K={w.K}; {el:.1f} s")
+    # throughput in the same unit: the step's algorithmic bytes, scaled to the rows sampled
+    byts = (sum(gemm_bytes(rows[M], w.N, w.K) for M in Ms) + sum(actq_bytes(rows[M], w.K) for M in Ms))
+    return {"value": byts * steps / el / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": sample,
+            "tops": 2 * sum(rows[M] for M in Ms) * w.N * w.K * steps / el / 1e12}
+
+
+# ---------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    Ms = list(w.Ms)
+    gb, ab, ops = step_accounting(w)
+    step_bytes = gb + ab
+
+    X, W = synth.make_workload(w)
+    qw, s_u8, a_u8, s_c = lq.lq_quantize_weights(W.to(dev))
+    wset_bytes = qw.numel() + s_u8.numel() + a_u8.numel() + 4 * s_c.numel()
+    n_sets = max(4, int(np.ceil(3 * L2_BYTES / wset_bytes)))
+    n_sets = min(n_sets, 64)
+    sets = [(qw, s_u8, a_u8, s_c)] + [(qw.clone(), s_u8.clone(), a_u8.clone(), s_c.clone())
+                                      for _ in range(n_sets - 1)]
+    Xd = X.to(dev)
+    Mx = max(Ms)
+    xq_buf = {M: torch.empty(M, w.K, dtype=torch.int8, device=dev) for M in Ms}
+    sx_buf = {M: torch.empty(M, dtype=torch.float32, device=dev) for M in Ms}
+    out_buf = {M: torch.empty(M, w.N, dtype=torch.bfloat16, device=dev) for M in Ms}
+    ws_need = max(lq.lq_w4a8_gemm_workspace_size(M, w.N, w.K) for M in Ms)
+    ws = torch.zeros(max(ws_need, 16), dtype=torch.uint8, device=dev)
+    # pinned host buffers for the end-to-end variant
+    X_host = X.pin_memory()
+    out_host = {M: torch.empty(M, w.N, dtype=torch.bfloat16).pin_memory() for M in Ms}
+    Xd_e2e = torch.empty_like(Xd)
+
+    stream = torch.cuda.Stream(dev)
+    counter = [0]
+
+    def step(events=None, e2e=False):
+        for M in Ms:
+            if e2e:
+                Xd_e2e[:M].copy_(X_host[:M], non_blocking=True)
+                src = Xd_e2e[:M]
+            else:
+                src = Xd[:M]
+            lq.lq_quantize_act(src, out=(xq_buf[M], sx_buf[M]))
+            wq = sets[counter[0] % n_sets]
+            counter[0] += 1
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True, external=True)
+                e1 = torch.cuda.Event(enable_timing=True, external=True)
+                e0.record()
+                lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=out_buf[M], workspace_buf=ws)
+                e1.record()
+                events.append((M, e0, e1))
+            else:
+                lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=out_buf[M], workspace_buf=ws)
+            if e2e:
+                out_host[M].copy_(out_buf[M], non_blocking=True)
+
+    def capture(nsteps, events=None, e2e=False):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(nsteps):
+                step(events, e2e)
+        return g
+
+    with torch.cuda.stream(stream):
+        # warm-up, eager, W steps (first launches also load the kernels)
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize(dev)
+        st = lq.lq_get_device_error(dev)
+        if st != 0:
+            raise RuntimeError(f"device error after warm-up: {st}")
+        gemm_events = []
+        g_timed = capture(args.steps)
+        g_instr = capture(args.steps, events=gemm_events)
+        g_soak = capture(max(1, min(args.steps, 50)))
+        g_e2e = None if args.no_e2e else capture(args.steps, e2e=True)
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    time.sleep(0.3)
+    t_load0 = time.time()
+    # untimed soak so the clocks settle and the sampler sees load
+    soak_end = time.time() + args.soak_s
+    while time.time() < soak_end:
+        g_soak.replay()
+        torch.cuda.synchronize(dev)
+
+    def timed(graph):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    with torch.cuda.stream(stream):
+        ms_total = timed(g_timed)
+        # the same K steps with CUDA events around every GEMM node: the GEMM's own
+        # duration per launch (events between kernels also cut the launch overlap,
+        # so these durations include each launch's full ramp-up and tail)
+        ms_instr = timed(g_instr)
+        gemm_ms = [(M, a.elapsed_time(b)) for M, a, b in gemm_events]
+        ms_e2e = timed(g_e2e) if g_e2e is not None else None
+    t_load1 = time.time()
+    clocks = sampler.stop(t_load0, t_load1) if sampler else None
+    st = lq.lq_get_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {st}")
+
+    K_ = args.steps
+    value = world * step_bytes * K_ / (ms_total * 1e-3) / 1e9
+    # dominant kernel: the GEMM, averaged over every launch in the timed region
+    per_M = {M: float(np.mean([t for m, t in gemm_ms if m == M])) for M in Ms}
+    gemm_time_s = sum(t for _, t in gemm_ms) * 1e-3
+    gemm_bytes_total = sum(gemm_bytes(M, w.N, w.K) for M, _ in gemm_ms)
+    achieved = gemm_bytes_total / gemm_time_s / 1e9
+    pk, pk_src = peaks()
+    hbm_peak = float(pk["hbm_gbs"])
+    int8_peak = INT8_OVER_BF16 * float(pk["bf16_tflops"])
+    gemm_launches = len(gemm_ms)
+    n_traffic = ncu_traffic(args.workload)
+    res = {
+        "metric": "W4A8 GEMM TOPS and HBM GB/s vs roofline at decode M=1-16 and prefill M=4096",
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K_,
+        "warmup": args.warmup,
+        "ms_per_step": ms_total / K_,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02) weights)",
+        "config": {
+            "workload": w.note, "M": Ms, "N": w.N, "K": w.K, "group": 64,
+            "step": "per M: lq_quantize_act + lq_w4a8_gemm (weights quantized offline)",
+            "l2": f"weights rotate over {n_sets} copies ({n_sets * wset_bytes / 2**20:.0f} MiB > 126 MB L2)",
+            "timing": "one CUDA graph of K steps between CUDA events; kernels launched with "
+                      "programmatic dependent launch",
+            "parallelism": f"replicas x{world}",
+        },
+        "tops": world * ops * K_ / (ms_total * 1e-3) / 1e12,
+        "gpu_launches": K_ * 2 * len(Ms),
+        "roofline": {
+            "bound": "hbm", "kernel": "w4a8_gemm_kernel", "achieved": achieved, "peak": hbm_peak,
+            "unit": "GB/s", "frac": achieved / hbm_peak,
+            "traffic": n_traffic,
+            "peak_source": pk_src,
+            "per_launch_us": {str(M): 1e3 * t for M, t in per_M.items()},
+            "launches": gemm_launches,
+            "how": "CUDA events around every GEMM node of a replay of the same K steps, "
+                   "right after the timed replay",
+            "instrumented_ms_per_step": ms_instr / args.steps,
+            "bytes_per_launch": {str(M): gemm_bytes(M, w.N, w.K) for M in Ms},
+        },
+        "clocks": clocks,
+    }
+    if ms_e2e is not None:
+        h2d = sum(M * w.K * 2 for M in Ms)
+        d2h = sum(M * w.N * 2 for M in Ms)
+        res["e2e"] = {"value": world * step_bytes * K_ / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": ms_e2e / K_,
+                      "how": "pinned host X -> device copy, quantize_act + gemm, device -> pinned host out, "
+                             "per M, same CUDA graph method"}
+    res["int8_peak_tops"] = int8_peak
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w)
+    return res
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    from w4a8_bit_weight_b200 import synth
+    if rank != 0:
+        return None
+    w = synth.WORKLOADS[args.workload]
+    steps = max(1, args.steps)
+    cb = cpu_baseline(w, budget_s=min(60.0, 2.0 + 0.1 * steps))
+    return {
+        "metric": "W4A8 GEMM TOPS and HBM GB/s vs roofline at decode M=1-16 and prefill M=4096",
+        "impl": "reference", "value": cb["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic", "config": {"workload": w.note, "M": list(w.Ms), "N": w.N, "K": w.K},
+        "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

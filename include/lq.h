@@ -116,11 +116,19 @@ LQ_API lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, 
  *   Requires group == 64, K % 128 == 0, 128 <= K <= 131072, N % 16 == 0,
  *   N >= 16; M == 0 is a no-op.
  *   workspace: device scratch of at least lq_w4a8_gemm_workspace_size(M,N,K)
- *   bytes (may be NULL when that is 0), 16-byte aligned, ZERO-FILLED by the
- *   caller before its first use.  Each call leaves it zero-filled again, so
- *   it can be reused by later calls on the same stream without clearing; two
- *   calls in flight at the same time must not share one.  After a call that
- *   ended in LQ_ERR_TIMEOUT the caller must clear it again.
+ *   bytes (may be NULL when that is 0, which the automatic schedule always
+ *   gives), 16-byte aligned, ZERO-FILLED by the caller before its first use.
+ *   Each call leaves it zero-filled again, so it can be reused by later calls
+ *   on the same stream without clearing; two calls in flight at the same time
+ *   must not share one.  After a call that ended in LQ_ERR_TIMEOUT the caller
+ *   must clear it again.
+ *   Launch overlap: the GEMM and lq_quantize_act are launched as programmatic
+ *   dependents of the preceding kernel in the stream (set LQ_PDL=0 in the
+ *   environment to disable).  The GEMM starts streaming qw, s_u8 and a_u8
+ *   before that kernel has finished, so those buffers must not be written by
+ *   a kernel that itself triggers early launch (this library's weight
+ *   quantizer does not); x_q, s_x, s_c and out are touched only after it has
+ *   completed.
  */
 LQ_API size_t lq_w4a8_gemm_workspace_size(int M, int N, int K);
 LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw,
@@ -130,19 +138,26 @@ LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t
 
 /*
  * lq_w4a8_gemm_ex -- lq_w4a8_gemm with the schedule chosen by the caller
- * (tests and tuning).  block_t: tokens per tile, one of 16, 32, 64, 128, 256,
- * or 0 for the automatic choice.  grid: number of CTAs, 0 for automatic; the
- * M x N x K work is cut into K-blocks of 128 and spread evenly over the CTAs
- * (stream-K), and tiles shared by several CTAs are reduced through the
- * workspace.  grid is clamped to the number of K-blocks of work.
- * out_i32: when nonzero, out receives the int32 accumulators acc[m,n]
- * instead of bf16 (bit-exact check of the contraction).
+ * (tests and tuning).
+ *   block_t: tokens per tile, one of 16, 32, 64, 128, 256; 0 = automatic.
+ *   split_k: CTAs per tile in a thread-block cluster, each summing one slice
+ *            of the K-blocks of 128; the partial sums are reduced through
+ *            distributed shared memory.  1, 2, 4 or 8 (8 only for block_t <=
+ *            32, 4 for block_t <= 64, 2 for block_t <= 128); 0 = automatic.
+ *   grid:    > 0 selects the stream-K schedule instead: the K-blocks of all
+ *            tiles are spread evenly over `grid` CTAs (clamped to the number
+ *            of K-blocks of work), and tiles shared by several CTAs are
+ *            reduced through the workspace.  Must be 0 when split_k > 0.
+ *   out_i32: when nonzero, out receives the int32 accumulators acc[m,n]
+ *            instead of bf16 (bit-exact check of the contraction).
+ * lq_w4a8_gemm_workspace_size_ex gives the workspace that schedule needs
+ * (nonzero only for stream-K schedules that share tiles).
  */
-LQ_API size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int grid);
+LQ_API size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int split_k, int grid);
 LQ_API lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw,
-                          const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c, void* out,
-                          int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
-                          int block_t, int grid, int out_i32, void* stream);
+                                 const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c, void* out,
+                                 int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
+                                 int block_t, int split_k, int grid, int out_i32, void* stream);
 
 /*
  * lq_w4a8_gemm_i32 -- the contraction only: acc[m,n] as int32 [M, N] (16-byte

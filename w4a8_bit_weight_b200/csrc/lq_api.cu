@@ -6,6 +6,7 @@
 
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -22,7 +23,6 @@ struct DeviceInfo {
   bool ready = false;
   bool sm100 = false;
   int sms = 0;
-  bool attr_set[16] = {};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -85,10 +85,11 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
 // ------------------------------------------------------------- schedule
 struct Schedule {
   int bt = 0;        // tokens per tile
+  int cs = 1;        // CTAs per tile in a cluster (split-K), 0 = stream-K
   int tiles_m = 0, tiles_n = 0, KB = 0;
   long long tiles = 0, U = 0;
   int grid = 0;
-  bool split = false;  // some tile is shared by several CTAs
+  bool split = false;  // stream-K: some tile is shared by several CTAs
   size_t ws_bytes = 0;
 };
 
@@ -101,7 +102,22 @@ int auto_block_t(int M) {
 
 bool valid_block_t(int bt) { return bt == 16 || bt == 32 || bt == 64 || bt == 128 || bt == 256; }
 
-Schedule make_schedule(int M, int N, int K, int block_t, int grid, int sms) {
+// largest cluster split instantiated for a tile width (shared-memory bound)
+int max_split(int bt) { return bt <= 32 ? 8 : bt == 64 ? 4 : bt == 128 ? 2 : 1; }
+
+bool valid_split(int bt, int cs) { return (cs == 1 || cs == 2 || cs == 4 || cs == 8) && cs <= max_split(bt); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("LQ_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// split_k > 0: cluster split of that many CTAs per tile; grid > 0: stream-K
+// over that many CTAs; both 0: automatic.
+Schedule make_schedule(int M, int N, int K, int block_t, int split_k, int grid, int sms) {
   Schedule s;
   s.bt = block_t ? block_t : auto_block_t(M);
   s.tiles_m = (M + s.bt - 1) / s.bt;
@@ -109,26 +125,36 @@ Schedule make_schedule(int M, int N, int K, int block_t, int grid, int sms) {
   s.KB = K / lq::kBlockK;
   s.tiles = (long long)s.tiles_m * s.tiles_n;
   s.U = s.tiles * s.KB;
-  long long g = grid;
-  if (g <= 0) {
-    // enough whole tiles for two waves: one CTA per tile; else spread K-blocks
-    // evenly over one CTA per SM (stream-K)
-    g = (s.tiles >= 2LL * sms) ? s.tiles : (long long)sms;
-  }
-  if (g > s.U) g = s.U;
-  if (g > INT_MAX) g = INT_MAX;
-  if (g < 1) g = 1;
-  s.grid = (int)g;
-  s.split = false;
-  for (long long c = 1; c < g; ++c)
-    if ((c * s.U / g) % s.KB != 0) {
-      s.split = true;
-      break;
+  if (grid > 0) {
+    long long g = grid;
+    if (g > s.U) g = s.U;
+    if (g > INT_MAX) g = INT_MAX;
+    s.cs = 0;
+    s.grid = (int)g;
+    for (long long c = 1; c < g; ++c)
+      if ((c * s.U / g) % s.KB != 0) {
+        s.split = true;
+        break;
+      }
+    if (s.split) {
+      const size_t acc = (size_t)s.tiles * s.bt * lq::kBlockN * sizeof(int32_t);
+      s.ws_bytes = acc + (((size_t)s.tiles * sizeof(unsigned) + 15) / 16) * 16;
     }
-  if (s.split) {
-    const size_t acc = (size_t)s.tiles * s.bt * lq::kBlockN * sizeof(int32_t);
-    s.ws_bytes = acc + (((size_t)s.tiles * sizeof(unsigned) + 15) / 16) * 16;
+    return s;
   }
+  int cs = split_k;
+  if (cs <= 0) {
+    // one wave: as many CTAs per tile as fit on the SMs, at least 4 K-blocks each
+    cs = 1;
+    for (int c = max_split(s.bt); c >= 2; c /= 2)
+      if (s.tiles * c <= sms && s.KB / c >= 4) {
+        cs = c;
+        break;
+      }
+  }
+  if (cs > s.KB) cs = 1;
+  s.cs = cs;
+  s.grid = (int)(s.tiles * cs);
   return s;
 }
 
@@ -140,41 +166,87 @@ lq_status check_gemm_shape(int M, int N, int K, int group) {
   return LQ_OK;
 }
 
-template <int BT, bool I32>
-lq_status launch_gemm_t(const Schedule& s, DeviceInfo* dev, const CUtensorMap& tx, const CUtensorMap& tw,
-                        const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
-  using C = lq::GemmCfg<BT>;
-  auto kern = lq::w4a8_gemm_kernel<BT, I32>;
-  const int slot = (BT == 16 ? 0 : BT == 32 ? 1 : BT == 64 ? 2 : BT == 128 ? 3 : 4) + (I32 ? 5 : 0);
-  if (!dev->attr_set[slot]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-      return LQ_ERR_CUDA;
-    dev->attr_set[slot] = true;
+template <typename Kern, typename... Args>
+lq_status launch_ex(Kern kern, int grid, int block, int smem, int cluster, bool pdl, cudaStream_t st,
+                    Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (cluster >= 2) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
   }
-  kern<<<s.grid, lq::kGemmThreads, C::kSmemBytes, st>>>(tx, tw, ts, ta, a);
-  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+template <int BT, int CS, bool I32>
+lq_status launch_gemm_t(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
+                        const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  using C = lq::GemmCfg<BT, CS>;
+  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32>;
+  // the attribute is per function and cheap; set it on every call so that any
+  // device current at call time is covered
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tw, ts, ta, a);
+}
+
+template <int BT, bool I32>
+lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
+                         const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  switch (s.cs) {
+    case 0: return launch_gemm_t<BT, 0, I32>(s, tx, tw, ts, ta, a, st);
+    case 1: return launch_gemm_t<BT, 1, I32>(s, tx, tw, ts, ta, a, st);
+    case 2:
+      if constexpr (BT <= 128) return launch_gemm_t<BT, 2, I32>(s, tx, tw, ts, ta, a, st);
+      break;
+    case 4:
+      if constexpr (BT <= 64) return launch_gemm_t<BT, 4, I32>(s, tx, tw, ts, ta, a, st);
+      break;
+    case 8:
+      if constexpr (BT <= 32) return launch_gemm_t<BT, 8, I32>(s, tx, tw, ts, ta, a, st);
+      break;
+  }
+  return LQ_ERR_INVALID_ARG;
 }
 
 template <bool I32>
-lq_status launch_gemm(const Schedule& s, DeviceInfo* dev, const CUtensorMap& tx, const CUtensorMap& tw,
-                      const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
+                      const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   switch (s.bt) {
-    case 16: return launch_gemm_t<16, I32>(s, dev, tx, tw, ts, ta, a, st);
-    case 32: return launch_gemm_t<32, I32>(s, dev, tx, tw, ts, ta, a, st);
-    case 64: return launch_gemm_t<64, I32>(s, dev, tx, tw, ts, ta, a, st);
-    case 128: return launch_gemm_t<128, I32>(s, dev, tx, tw, ts, ta, a, st);
-    case 256: return launch_gemm_t<256, I32>(s, dev, tx, tw, ts, ta, a, st);
+    case 16: return launch_gemm_bt<16, I32>(s, tx, tw, ts, ta, a, st);
+    case 32: return launch_gemm_bt<32, I32>(s, tx, tw, ts, ta, a, st);
+    case 64: return launch_gemm_bt<64, I32>(s, tx, tw, ts, ta, a, st);
+    case 128: return launch_gemm_bt<128, I32>(s, tx, tw, ts, ta, a, st);
+    case 256: return launch_gemm_bt<256, I32>(s, tx, tw, ts, ta, a, st);
   }
   return LQ_ERR_INVALID_ARG;
 }
 
 lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                     const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
-                    void* workspace, size_t ws_bytes, int block_t, int grid, bool out_i32, void* stream) {
+                    void* workspace, size_t ws_bytes, int block_t, int split_k, int grid, bool out_i32,
+                    void* stream) {
   lq_status st = check_gemm_shape(M, N, K, group);
   if (st != LQ_OK) return st;
   if (block_t != 0 && !valid_block_t(block_t)) return LQ_ERR_INVALID_ARG;
-  if (grid < 0) return LQ_ERR_INVALID_ARG;
+  if (grid < 0 || split_k < 0 || (grid > 0 && split_k > 0)) return LQ_ERR_INVALID_ARG;
+  if (split_k > 0 && !valid_split(block_t ? block_t : auto_block_t(M > 0 ? M : 1), split_k))
+    return LQ_ERR_INVALID_ARG;
   if (M == 0) return LQ_OK;
   if (!x_q || !qw || !s_u8 || !a_u8 || !out || (!out_i32 && (!s_x || !s_c))) return LQ_ERR_INVALID_ARG;
   if (!aligned(x_q, 16) || !aligned(qw, 16) || !aligned(s_u8, 16) || !aligned(a_u8, 16) ||
@@ -183,7 +255,7 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
-  const Schedule s = make_schedule(M, N, K, block_t, grid, dev->sms);
+  const Schedule s = make_schedule(M, N, K, block_t, split_k, grid, dev->sms);
   if (s.split) {
     if (!workspace || ws_bytes < s.ws_bytes) return LQ_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return LQ_ERR_MISALIGNED;
@@ -213,8 +285,7 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   a.KB = s.KB;
   a.U = s.U;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return out_i32 ? launch_gemm<true>(s, dev, tx, tw, ts, ta, a, cs)
-                 : launch_gemm<false>(s, dev, tx, tw, ts, ta, a, cs);
+  return out_i32 ? launch_gemm<true>(s, tx, tw, ts, ta, a, cs) : launch_gemm<false>(s, tx, tw, ts, ta, a, cs);
 }
 
 }  // namespace
@@ -260,44 +331,44 @@ lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, float* 
   DeviceInfo* dev = nullptr;
   lq_status st = current_device(&dev);
   if (st != LQ_OK) return st;
-  lq::quantize_act_kernel<<<M, lq::kQuantActThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(X_bf16), K, x_q, s_x);
-  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+  return launch_ex(lq::quantize_act_kernel, M, lq::kQuantActThreads, 0, 1, pdl_enabled(),
+                   static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(X_bf16), K, x_q, s_x);
 }
 
-size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int grid) {
+size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int split_k, int grid) {
   if (check_gemm_shape(M, N, K, LQ_GROUP) != LQ_OK || M == 0) return 0;
   if (block_t != 0 && !valid_block_t(block_t)) return 0;
+  if (grid < 0 || split_k < 0) return 0;
   DeviceInfo* dev = nullptr;
   int sms = 148;
   if (current_device(&dev) == LQ_OK) sms = dev->sms;
-  return make_schedule(M, N, K, block_t, grid, sms).ws_bytes;
+  return make_schedule(M, N, K, block_t, split_k, grid, sms).ws_bytes;
 }
 
 size_t lq_w4a8_gemm_workspace_size(int M, int N, int K) {
-  return lq_w4a8_gemm_workspace_size_ex(M, N, K, 0, 0);
+  return lq_w4a8_gemm_workspace_size_ex(M, N, K, 0, 0, 0);
 }
 
 lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                           const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
-                          void* workspace, size_t workspace_bytes, int block_t, int grid, int out_i32,
-                          void* stream) {
+                          void* workspace, size_t workspace_bytes, int block_t, int split_k, int grid,
+                          int out_i32, void* stream) {
   return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out, M, N, K, group, workspace, workspace_bytes, block_t,
-                   grid, out_i32 != 0, stream);
+                   split_k, grid, out_i32 != 0, stream);
 }
 
 lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                        const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K, int group,
                        void* workspace, size_t workspace_bytes, void* stream) {
   return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes, 0, 0,
-                   false, stream);
+                   0, false, stream);
 }
 
 lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8,
                            int32_t* acc, int M, int N, int K, int group, void* workspace,
                            size_t workspace_bytes, void* stream) {
   return gemm_impl(x_q, nullptr, qw, s_u8, a_u8, nullptr, acc, M, N, K, group, workspace, workspace_bytes, 0,
-                   0, true, stream);
+                   0, 0, true, stream);
 }
 
 lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8, int N, int K,

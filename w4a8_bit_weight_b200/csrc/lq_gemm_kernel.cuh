@@ -9,7 +9,7 @@
 // shared-memory bandwidth is left to the activation tiles and the packed
 // weights.
 //
-// Warp roles (192 threads, one CTA per SM):
+// Warp roles (192 threads):
 //   warp 0     TMA producer: packed u4 weights, u8 scale/offset tiles and
 //              int8 activation tiles into a ring of shared-memory stages.
 //   warp 1     allocates TMEM; one thread issues tcgen05.mma kind::i8.
@@ -17,13 +17,26 @@
 //              one XOR per four weights) into the TMEM A slot of the stage,
 //              then the epilogue: int32 accumulators -> scales -> bf16.
 //
-// Schedule (stream-K): the M x N x K work is cut into units of one tile x one
-// K-block of 128; CTA c takes units [c*U/G, (c+1)*U/G).  A tile whose units
-// all belong to one CTA is written directly; a tile shared by several CTAs is
-// summed in an int32 workspace with atomic adds, and the CTA that arrives last
-// (atomic ticket) applies the epilogue and restores the workspace and the
-// ticket to zero.  Integer sums are order-independent, so the result is
-// bit-identical either way.
+// Schedules (CS template parameter):
+//   CS >= 1  split-K inside a thread-block cluster of CS CTAs: the cluster
+//            owns one 128-row x BT-token tile, CTA rank r takes the r-th
+//            slice of the K-blocks.  The non-leader CTAs write their int32
+//            partial sums into the leader's shared memory (DSMEM) and arrive
+//            on its mbarrier; the leader adds them and runs the epilogue.
+//            CS = 1 is the plain one-CTA-per-tile schedule.
+//   CS == 0  stream-K over any grid: the M x N x K work is cut into units of
+//            one tile x one K-block of 128; CTA c takes units
+//            [c*U/G, (c+1)*U/G).  Tiles shared by several CTAs are summed in
+//            an int32 workspace with atomic adds; the CTA that arrives last
+//            (atomic ticket) applies the epilogue and restores the workspace
+//            and the ticket to zero.
+// Integer sums are order-independent, so every schedule gives bit-identical
+// results.
+//
+// Programmatic dependent launch: the producer issues the weight loads of the
+// first stages before griddepcontrol.wait (weights are never written by the
+// kernel this launch overlaps), and the activation loads after it; the
+// epilogue waits before it reads scales or writes the output.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -35,36 +48,41 @@ namespace lq {
 constexpr int kBlockN = 128;        // weight rows per tile (MMA M)
 constexpr int kBlockK = 128;        // K per pipeline stage (two groups of 64)
 constexpr int kGemmThreads = 192;
-constexpr int kTmemCols = 512;
 
 __host__ __device__ constexpr int round_up_c(int x, int a) { return (x + a - 1) / a * a; }
+__host__ __device__ constexpr int max_c(int a, int b) { return a > b ? a : b; }
 
-template <int BT>
+template <int BT, int CS>
 struct GemmCfg {
   static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128 || BT == 256, "tokens per tile");
-  static constexpr int kStages = BT == 256 ? 5 : 8;
+  static_assert(CS >= 0 && CS <= 8, "cluster size");
+  static constexpr int kStages = BT <= 64 ? 6 : (BT == 128 ? (CS >= 2 ? 6 : 8) : 5);
   static constexpr int kXBytes = BT * kBlockK;             // int8 activation tile, 128-byte rows
   static constexpr int kWBytes = kBlockN * kBlockK / 2;    // packed u4 weight tile, 64-byte rows
   static constexpr int kSABytes = 2 * kBlockN;             // 2 groups x 128 rows of u8
   static constexpr int kStageBytes = round_up_c(kXBytes + kWBytes + 2 * kSABytes, 1024);
   static constexpr uint32_t kTxBytes = kXBytes + kWBytes + 2 * kSABytes;
+  static constexpr uint32_t kTxWeights = kWBytes + 2 * kSABytes;
   static constexpr int kAccCols = BT < 32 ? 32 : BT;      // int32 accumulator columns
+  static constexpr int kTmemCols = (kAccCols + kStages * 32 <= 256) ? 256 : 512;
+  static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * BT * kBlockN * 4 : 0;  // DSMEM partials
   static constexpr int kBarBytes = 256;
-  // at least 120 KB so that two CTAs never share an SM (each holds 512 TMEM columns)
-  static constexpr int kSmemBytes =
-      round_up_c(kStages * kStageBytes + kBarBytes, 1024) + 1024 > 122880
-          ? round_up_c(kStages * kStageBytes + kBarBytes, 1024) + 1024
-          : 122880;
+  static constexpr int kUsed = kStages * kStageBytes + kRedBytes + kBarBytes + 1024;  // + alignment slack
+  // Shared memory also bounds how many CTAs share an SM: a 512-column CTA
+  // takes at least 120 KB (one per SM), a 256-column CTA at least 80 KB (at
+  // most two per SM), so co-resident CTAs never exceed the 512 TMEM columns.
+  static constexpr int kSmemBytes = max_c(round_up_c(kUsed, 1024), kTmemCols == 512 ? 122880 : 81920);
   static_assert(kAccCols + kStages * 32 <= kTmemCols, "TMEM budget");
-  static_assert(3 * kStages * 8 + 4 * 8 + 16 <= kBarBytes, "barrier area");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(3 * kStages * 8 + 5 * 8 + 16 <= kBarBytes, "barrier area");
 };
 
 struct GemmArgs {
   const float* s_x;
   const float* s_c;
   void* out;             // bf16 [M, N] or int32 [M, N]
-  int32_t* ws;           // [tiles][BT][128] int32, zero between calls
-  unsigned int* ticket;  // [tiles], zero between calls
+  int32_t* ws;           // stream-K only: [tiles][BT][128] int32, zero between calls
+  unsigned int* ticket;  // stream-K only: [tiles], zero between calls
   int M, N, K;
   int tiles_m, KB;
   long long U;           // units = tiles * KB
@@ -95,27 +113,46 @@ __device__ __forceinline__ void store_out(const GemmArgs& p, int m, int n, int32
   }
 }
 
-template <int BT, bool OUT_I32>
+// Reads CH accumulator columns [c0, c0+CH) of this warp's 32 TMEM lanes.
+template <int CH>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&v)[32]) {
+  if constexpr (CH == 16) {
+    uint32_t v16[16];
+    tmem_ld_32x32b_x16(taddr, v16);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = v16[i];
+  } else {
+    tmem_ld_32x32b_x32(taddr, v);
+    tmem_ld_wait();
+  }
+}
+
+template <int BT, int CS, bool OUT_I32>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
                      const GemmArgs p) {
-  using C = GemmCfg<BT>;
+  using C = GemmCfg<BT, CS>;
   constexpr int S = C::kStages;
+  constexpr int CH = BT < 32 ? BT : 32;  // accumulator columns per TMEM load
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  int32_t* red = reinterpret_cast<int32_t*>(smem + S * C::kStageBytes);  // [CS-1][BT][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kRedBytes);
   uint64_t* afull = full + S;
   uint64_t* empty = afull + S;
   uint64_t* accfull = empty + S;
   uint64_t* drain = accfull + 1;
   uint64_t* grp = drain + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(grp + 1);
+  uint64_t* redbar = grp + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t crank = CS >= 2 ? cluster_ctarank() : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -126,6 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(accfull, 1);
     mbar_init(drain, 1);
     mbar_init(grp, 4);
+    mbar_init(redbar, CS >= 2 ? (CS - 1) * 128 : 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -135,99 +173,145 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tm_a);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Cluster barrier, first half: this CTA's barriers are initialized.  The
+  // second half is waited on only before a remote arrive (and at teardown).
+  if constexpr (CS >= 2) cluster_arrive();
+  bool cl_waited = false;
 
+  // this CTA's range of units (tile x K-block)
+  const int KB = p.KB;
+  long long u_begin, u_end;
   const long long U = p.U;
   const long long G = gridDim.x;
-  const long long u_begin = (long long)blockIdx.x * U / G;
-  const long long u_end = ((long long)blockIdx.x + 1) * U / G;
-  const int KB = p.KB;
+  if constexpr (CS >= 1) {
+    const long long t = blockIdx.x / CS;
+    const int r = (int)(blockIdx.x % CS);
+    u_begin = t * KB + (long long)r * KB / CS;
+    u_end = t * KB + (long long)(r + 1) * KB / CS;
+  } else {
+    u_begin = (long long)blockIdx.x * U / G;
+    u_end = ((long long)blockIdx.x + 1) * U / G;
+  }
 
+  // Producer and MMA warps run their loops with all 32 lanes (one lane issues),
+  // so every warp stays converged up to the CTA barrier at teardown.
+  const bool leader = (lane == 0);
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_stream = l2_policy_evict_first();  // weights: read once
-      const uint64_t pol_keep = l2_policy_evict_last();     // activations: re-read per weight tile
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0, issued_par = 0;  // per stage: load in flight, its phase parity
-      for (long long u = u_begin; u < u_end;) {
-        const int t = (int)(u / KB);
-        const int kb0 = (int)(u % KB);
-        const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
-        const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
-          uint8_t* sb = smem + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
-          tma_load_2d(sb, &tm_x, &full[stage], kb * kBlockK, tile_m * BT, pol_keep);
-          tma_load_2d(sb + C::kXBytes, &tm_w, &full[stage], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
-          tma_load_2d(sb + C::kXBytes + C::kWBytes, &tm_s, &full[stage], tile_n * kBlockN, kb * 2, pol_stream);
-          tma_load_2d(sb + C::kXBytes + C::kWBytes + C::kSABytes, &tm_a, &full[stage], tile_n * kBlockN, kb * 2,
-                      pol_stream);
+    uint64_t pol_stream = 0, pol_keep = 0;
+    if (leader) {
+      pol_stream = l2_policy_evict_first();  // weights: read once
+      pol_keep = l2_policy_evict_last();     // activations: re-read per weight tile
+    }
+    // weights of the first stages do not depend on the preceding kernel
+    const int t0 = (int)(u_begin / KB);
+    const int kbf = (int)(u_begin % KB);
+    const int P = (int)min((long long)S, min((long long)(KB - kbf), u_end - u_begin));
+    const int tn0 = t0 / p.tiles_m, tm0 = t0 % p.tiles_m;
+    if (leader) {
+      for (int i = 0; i < P; ++i) {
+        uint8_t* sb = smem + i * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[i], C::kTxBytes);
+        tma_load_2d(sb + C::kXBytes, &tm_w, &full[i], (kbf + i) * (kBlockK / 2), tn0 * kBlockN, pol_stream);
+        tma_load_2d(sb + C::kXBytes + C::kWBytes, &tm_s, &full[i], tn0 * kBlockN, (kbf + i) * 2, pol_stream);
+        tma_load_2d(sb + C::kXBytes + C::kWBytes + C::kSABytes, &tm_a, &full[i], tn0 * kBlockN, (kbf + i) * 2,
+                    pol_stream);
+      }
+    }
+    griddep_wait();
+    if (leader)
+      for (int i = 0; i < P; ++i)
+        tma_load_2d(smem + i * C::kStageBytes, &tm_x, &full[i], (kbf + i) * kBlockK, tm0 * BT, pol_keep);
+    __syncwarp();
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = P >= 32 ? 0xffffffffu : ((1u << P) - 1u), issued_par = 0;
+    int it = 0;
+    for (long long u = u_begin; u < u_end;) {
+      const int t = (int)(u / KB);
+      const int kb0 = (int)(u % KB);
+      const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+      const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        if (it >= P) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1u, abort_flag))) goto producer_done;
+          if (leader) {
+            uint8_t* sb = smem + stage * C::kStageBytes;
+            mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
+            tma_load_2d(sb, &tm_x, &full[stage], kb * kBlockK, tile_m * BT, pol_keep);
+            tma_load_2d(sb + C::kXBytes, &tm_w, &full[stage], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
+            tma_load_2d(sb + C::kXBytes + C::kWBytes, &tm_s, &full[stage], tile_n * kBlockN, kb * 2, pol_stream);
+            tma_load_2d(sb + C::kXBytes + C::kWBytes + C::kSABytes, &tm_a, &full[stage], tile_n * kBlockN, kb * 2,
+                        pol_stream);
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      u += kb1 - kb0;
+    }
+  producer_done:
+    if (leader && *abort_flag) {
+      // never leave a bulk copy in flight into shared memory that is about to be released
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) {
+          const uint32_t a = smem_u32(&full[s]);
+          const unsigned long long t0w = globaltimer();
+          while (!mbar_try_wait(a, (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
           }
         }
-        u += kb1 - kb0;
-      }
-    producer_done:
-      if (*abort_flag) {
-        // never leave a bulk copy in flight into shared memory that is about to be released
-        for (int s = 0; s < S; ++s)
-          if (issued & (1u << s)) {
-            const uint32_t a = smem_u32(&full[s]);
-            const unsigned long long t0 = globaltimer();
-            while (!mbar_try_wait(a, (issued_par >> s) & 1u) && globaltimer() - t0 < 100000000ull) {
-            }
-          }
-      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(BT);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool any = false;
-      for (long long u = u_begin; u < u_end;) {
-        const int kb0 = (int)(u % KB);
-        const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&afull[stage], phase, abort_flag)) goto mma_done;
-          tc_fence_after();
+    constexpr uint32_t idesc = idesc_i8(BT);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool any = false;
+    for (long long u = u_begin; u < u_end;) {
+      const int kb0 = (int)(u % KB);
+      const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&afull[stage], phase, abort_flag))) goto mma_done;
+        tc_fence_after();
+        if (leader) {
           const uint64_t bdesc = smem_desc_k_sw128(smem_u32(smem + stage * C::kStageBytes));
           const uint32_t a_col = tmem_base + C::kAccCols + stage * 32;
 #pragma unroll
           for (int j = 0; j < kBlockK / 32; ++j)
             mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb > kb0 || j > 0) ? 1u : 0u);
           tc_commit(&empty[stage]);
-          any = true;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
-        tc_commit(accfull);
-        u += kb1 - kb0;
+        __syncwarp();
+        any = true;
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
-    mma_done:
-      if (any) {
-        // all issued MMAs have finished before TMEM is released
-        tc_commit(drain);
-        const uint32_t a = smem_u32(drain);
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(a, 0) && globaltimer() - t0 < 100000000ull) {
-        }
+      if (leader) tc_commit(accfull);
+      __syncwarp();
+      u += kb1 - kb0;
+    }
+    // the next kernel in the stream may start its prologue
+    griddep_launch_dependents();
+  mma_done:
+    if (leader && any) {
+      // all issued MMAs have finished before TMEM is released
+      tc_commit(drain);
+      const uint32_t a = smem_u32(drain);
+      const unsigned long long t0w = globaltimer();
+      while (!mbar_try_wait(a, 0) && globaltimer() - t0w < 100000000ull) {
       }
     }
   } else {
@@ -238,6 +322,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int sw = (r >> 1) & 3;        // 64-byte swizzle of this row's 16-byte chunks
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0, grp_phase = 0;
+    bool waited_dep = false;
+    bool red_done = (CS < 2 || crank != 0);
     for (long long u = u_begin; u < u_end;) {
       const int t = (int)(u / KB);
       const int kb0 = (int)(u % KB);
@@ -276,6 +362,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
 
       // ------------------------------------------------------- epilogue
+      if (!waited_dep) {
+        griddep_wait();  // scales and the output may belong to the preceding kernel
+        waited_dep = true;
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
       acc_phase ^= 1u;
       tc_fence_after();
@@ -285,72 +375,119 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool n_ok = n < p.N;
         const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
         const bool whole = (kb0 == 0 && kb1 == KB);
-        int32_t* ws_tile = p.ws + (size_t)t * BT * kBlockN;
-        constexpr int CH = BT < 32 ? BT : 32;
+        if constexpr (CS >= 2) {
+          // ----------------------------------------- cluster split-K (DSMEM)
+          if (crank != 0) {
+            // the leader's barrier is initialized once the whole cluster has arrived
+            cluster_wait();
+            cl_waited = true;
+            // partial sums -> leader's shared memory, then one release-arrive per thread
+            const uint32_t dst = mapa_shared(smem_u32(red + (size_t)(crank - 1) * BT * kBlockN + r), 0);
 #pragma unroll 1
-        for (int cc = 0; cc < BT / CH; ++cc) {
-          uint32_t v[32];
-          if constexpr (CH == 16) {
-            uint32_t v16[16];
-            tmem_ld_32x32b_x16(t_lane + cc * CH, v16);
-            tmem_ld_wait();
+            for (int cc = 0; cc < BT / CH; ++cc) {
+              uint32_t v[32];
+              tmem_load_cols<CH>(t_lane + cc * CH, v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = v16[i];
+              for (int i = 0; i < CH; ++i) st_cluster_u32(dst + (uint32_t)((cc * CH + i) * kBlockN * 4), v[i]);
+            }
+            tc_fence_before();
+            mbar_arrive_remote(mapa_shared(smem_u32(redbar), 0));
           } else {
-            tmem_ld_32x32b_x32(t_lane + cc * CH, v);
-            tmem_ld_wait();
-          }
+            if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
+            red_done = true;
+#pragma unroll 1
+            for (int cc = 0; cc < BT / CH; ++cc) {
+              uint32_t v[32];
+              tmem_load_cols<CH>(t_lane + cc * CH, v);
 #pragma unroll
-          for (int i = 0; i < CH; ++i) {
-            const int ml = cc * CH + i;
-            const int m = m0 + ml;
-            if (m < p.M) {
-              if (whole) {
-                if (n_ok) store_out<OUT_I32>(p, m, n, (int32_t)v[i], sc);
-              } else {
-                atomicAdd(ws_tile + ml * kBlockN + r, (int32_t)v[i]);
+              for (int i = 0; i < CH; ++i) {
+                const int ml = cc * CH + i;
+                int32_t acc = (int32_t)v[i];
+#pragma unroll
+                for (int j = 0; j < CS - 1; ++j) acc += red[((size_t)j * BT + ml) * kBlockN + r];
+                const int m = m0 + ml;
+                if (m < p.M && n_ok) store_out<OUT_I32>(p, m, n, acc, sc);
+              }
+            }
+            tc_fence_before();
+          }
+        } else {
+          int32_t* ws_tile = p.ws + (size_t)t * BT * kBlockN;
+#pragma unroll 1
+          for (int cc = 0; cc < BT / CH; ++cc) {
+            uint32_t v[32];
+            tmem_load_cols<CH>(t_lane + cc * CH, v);
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+              const int ml = cc * CH + i;
+              const int m = m0 + ml;
+              if (m < p.M) {
+                if (whole) {
+                  if (n_ok) store_out<OUT_I32>(p, m, n, (int32_t)v[i], sc);
+                } else {
+                  atomicAdd(ws_tile + ml * kBlockN + r, (int32_t)v[i]);
+                }
               }
             }
           }
-        }
-        tc_fence_before();
-        if (!whole) {
-          __threadfence();
-          if (!group_sync(grp, grp_phase, abort_flag)) goto epi_done;
-          if (warp == 2 && lane == 0) {
-            const long long first = cta_of_unit((long long)t * KB, U, G);
-            const long long last = cta_of_unit((long long)t * KB + KB - 1, U, G);
-            const unsigned contributors = (unsigned)(last - first + 1);
-            const unsigned prev = atomicAdd(p.ticket + t, 1u);
-            *last_flag = (prev == contributors - 1) ? 1 : 0;
-          }
-          if (!group_sync(grp, grp_phase, abort_flag)) goto epi_done;
-          if (*last_flag) {
+          tc_fence_before();
+          if (CS == 0 && !whole) {
+            // ------------------------------------- stream-K: last arriver finishes
             __threadfence();
-            for (int ml = 0; ml < BT; ++ml) {
-              const int m = m0 + ml;
-              if (m >= p.M) break;
-              int32_t* cell = ws_tile + ml * kBlockN + r;
-              const int32_t acc = __ldcg(cell);
-              *cell = 0;
-              if (n_ok) store_out<OUT_I32>(p, m, n, acc, sc);
+            if (!group_sync(grp, grp_phase, abort_flag)) goto epi_done;
+            if (warp == 2 && lane == 0) {
+              const long long first = cta_of_unit((long long)t * KB, U, G);
+              const long long last = cta_of_unit((long long)t * KB + KB - 1, U, G);
+              const unsigned contributors = (unsigned)(last - first + 1);
+              const unsigned prev = atomicAdd(p.ticket + t, 1u);
+              *last_flag = (prev == contributors - 1) ? 1 : 0;
             }
-            if (warp == 2 && lane == 0) p.ticket[t] = 0u;
+            if (!group_sync(grp, grp_phase, abort_flag)) goto epi_done;
+            if (*last_flag) {
+              __threadfence();
+              const int mrows = min(BT, p.M - m0);
+#pragma unroll 1
+              for (int mb = 0; mb < mrows; mb += 16) {
+                int32_t vals[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  vals[i] = (mb + i < mrows) ? __ldcg(ws_tile + (mb + i) * kBlockN + r) : 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  if (mb + i < mrows) {
+                    ws_tile[(mb + i) * kBlockN + r] = 0;
+                    if (n_ok) store_out<OUT_I32>(p, m0 + mb + i, n, vals[i], sc);
+                  }
+              }
+              if (warp == 2 && lane == 0) p.ticket[t] = 0u;
+            }
           }
         }
       }
       u += kb1 - kb0;
     }
-  epi_done:;
+  epi_done:
+    if (!red_done) {
+      // leader on an error path: non-leaders may still be writing into this
+      // CTA's shared memory; wait (bounded) for their arrivals before leaving
+      const uint32_t a = smem_u32(redbar);
+      const unsigned long long t0w = globaltimer();
+      while (!mbar_try_wait_cluster(a, 0) && globaltimer() - t0w < 100000000ull) {
+      }
+    }
   }
 
   // ---------------------------------------------------------------- teardown
+  __syncwarp();
+  if constexpr (CS >= 2) {
+    if (!cl_waited) cluster_wait();  // every thread completes the cluster barrier once
+  }
   tc_fence_before();
-  __syncthreads();
+  cta_barrier_unaligned();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 

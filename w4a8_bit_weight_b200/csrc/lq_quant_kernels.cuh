@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(kQuantActThreads) quantize_act_kernel(const ui
                                                                         int K, int8_t* __restrict__ x_q,
                                                                         float* __restrict__ s_x) {
   __shared__ float red[32];
+  griddep_launch_dependents();  // the GEMM that follows may start streaming its weights
+  griddep_wait();               // X may be the output of the preceding kernel
   const int m = blockIdx.x;
   const uint16_t* row = X + (size_t)m * K;
   float amax = 0.0f;
