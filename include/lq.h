@@ -136,28 +136,43 @@ LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t
                        void* out_bf16, int M, int N, int K, int group, void* workspace,
                        size_t workspace_bytes, void* stream);
 
+/* Schedules of lq_w4a8_gemm_ex. */
+#define LQ_SCHED_AUTO 0       /* what lq_w4a8_gemm uses */
+#define LQ_SCHED_TILES 1      /* one cluster of split_k CTAs per tile */
+#define LQ_SCHED_PERSISTENT 2 /* grid CTAs loop over 128-token tiles */
+#define LQ_SCHED_STREAMK 3    /* grid CTAs share the K-blocks of all tiles */
+
 /*
  * lq_w4a8_gemm_ex -- lq_w4a8_gemm with the schedule chosen by the caller
- * (tests and tuning).
- *   block_t: tokens per tile, one of 16, 32, 64, 128, 256; 0 = automatic.
- *   split_k: CTAs per tile in a thread-block cluster, each summing one slice
- *            of the K-blocks of 128; the partial sums are reduced through
- *            distributed shared memory.  1, 2, 4 or 8 (8 only for block_t <=
- *            32, 4 for block_t <= 64, 2 for block_t <= 128); 0 = automatic.
- *   grid:    > 0 selects the stream-K schedule instead: the K-blocks of all
- *            tiles are spread evenly over `grid` CTAs (clamped to the number
- *            of K-blocks of work), and tiles shared by several CTAs are
- *            reduced through the workspace.  Must be 0 when split_k > 0.
- *   out_i32: when nonzero, out receives the int32 accumulators acc[m,n]
- *            instead of bf16 (bit-exact check of the contraction).
+ * (tests and tuning).  Same result for every schedule (integer sums).
+ *   block_t:  tokens per tile, one of 16, 32, 64, 128, 256; 0 = automatic
+ *             (LQ_SCHED_PERSISTENT accepts only 0 or 128).
+ *   schedule: LQ_SCHED_AUTO: block_t may be set, split_k and grid must be 0.
+ *             LQ_SCHED_TILES: each tile of 128 weight rows x block_t tokens is
+ *               computed by a thread-block cluster of split_k CTAs, each
+ *               summing one slice of the K-blocks of 128; partial sums are
+ *               reduced through distributed shared memory.  split_k is 1, 2,
+ *               4 or 8 (8 only for block_t <= 32, 4 for block_t <= 64, 2 for
+ *               block_t <= 128, 1 for 256); 0 = automatic.  grid must be 0.
+ *             LQ_SCHED_PERSISTENT: grid CTAs (0 = one per SM) loop over the
+ *               tiles, overlapping each tile's epilogue with the next tile's
+ *               main loop.  split_k must be 0.
+ *             LQ_SCHED_STREAMK: the K-blocks of all tiles are spread evenly
+ *               over grid CTAs (0 = one per SM; clamped to the number of
+ *               K-blocks of work); tiles shared by several CTAs are reduced
+ *               through the workspace.  split_k must be 0.
+ *   out_i32:  when nonzero, out receives the int32 accumulators acc[m,n]
+ *             instead of bf16 (bit-exact check of the contraction).
  * lq_w4a8_gemm_workspace_size_ex gives the workspace that schedule needs
- * (nonzero only for stream-K schedules that share tiles).
+ * (nonzero only for LQ_SCHED_STREAMK when tiles are shared).
  */
-LQ_API size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int split_k, int grid);
+LQ_API size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int schedule, int split_k,
+                                             int grid);
 LQ_API lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw,
                                  const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c, void* out,
                                  int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
-                                 int block_t, int split_k, int grid, int out_i32, void* stream);
+                                 int block_t, int schedule, int split_k, int grid, int out_i32,
+                                 void* stream);
 
 /*
  * lq_w4a8_gemm_i32 -- the contraction only: acc[m,n] as int32 [M, N] (16-byte

@@ -35,8 +35,9 @@ ODD = P((1 << 20) + 8)
 
 
 def gemm(lib, M=16, N=256, K=512, group=64, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=GOOD, sc=GOOD, out=GOOD,
-         bt=0, split=0, grid=0):
-    return lib.lq_w4a8_gemm_ex(x, sx, qw, s, a, sc, out, M, N, K, group, None, 0, bt, split, grid, 0, None)
+         bt=0, sched=0, split=0, grid=0):
+    return lib.lq_w4a8_gemm_ex(x, sx, qw, s, a, sc, out, M, N, K, group, None, 0, bt, sched, split, grid, 0,
+                               None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -47,10 +48,14 @@ def gemm(lib, M=16, N=256, K=512, group=64, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=
     (dict(sx=P(0)), 1), (dict(sc=P(0)), 1),
     (dict(x=ODD), 3), (dict(qw=ODD), 3), (dict(s=ODD), 3), (dict(a=ODD), 3), (dict(out=ODD), 3),
     (dict(sx=P((1 << 20) + 2)), 3),
-    (dict(bt=48), 1), (dict(grid=-1), 1), (dict(split=-1), 1), (dict(split=3), 1),
-    (dict(split=2, grid=4), 1),           # cluster split and stream-K are exclusive
-    (dict(bt=64, split=8), 1),            # split 8 only for tiles of <= 32 tokens
-    (dict(bt=256, split=2), 1),           # 256-token tiles are never split
+    (dict(bt=48), 1), (dict(sched=4), 1), (dict(sched=-1), 1),
+    (dict(sched=3, grid=-1), 1), (dict(sched=1, split=-1), 1), (dict(sched=1, split=3), 1),
+    (dict(split=2), 1), (dict(grid=4), 1),        # the automatic schedule takes no split or grid
+    (dict(sched=1, split=2, grid=4), 1),          # a cluster split has no grid
+    (dict(sched=3, split=2, grid=4), 1),          # stream-K has no cluster split
+    (dict(sched=1, bt=64, split=8), 1),           # split 8 only for tiles of <= 32 tokens
+    (dict(sched=1, bt=256, split=2), 1),          # 256-token tiles are never split
+    (dict(sched=2, bt=64), 1),                    # the persistent schedule uses 128-token tiles
 ])
 def test_gemm_rejects_before_launch(lib, kw, code):
     assert gemm(lib, **kw) == code
@@ -84,8 +89,9 @@ def test_workspace_size_rules(lib):
     assert lib.lq_w4a8_gemm_workspace_size(0, 256, 512) == 0
     # the automatic schedule and cluster splits never need a workspace
     assert lib.lq_w4a8_gemm_workspace_size(16, 4096, 4096) == 0
-    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 4, 0) == 0
+    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 1, 4, 0) == 0
+    assert lib.lq_w4a8_gemm_workspace_size_ex(4096, 4096, 4096, 0, 2, 0, 0) == 0
     # stream-K with one CTA per tile (grid = tiles): no tile is shared, no workspace
-    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 0, 2) == 0
+    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 3, 0, 2) == 0
     # 3 CTAs over 2 tiles x 4 K-blocks: split tiles need [tiles][16][128] int32 + tickets
-    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 0, 3) == 2 * 16 * 128 * 4 + 16
+    assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 3, 0, 3) == 2 * 16 * 128 * 4 + 16

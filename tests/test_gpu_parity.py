@@ -104,48 +104,54 @@ def test_dequant_identity_all_codes_on_gpu():
 # GEMM: int32 bit-exact and bf16 within 1 ulp, across schedules
 # ----------------------------------------------------------------------------
 
+T, P, SK = lq.SCHED_TILES, lq.SCHED_PERSISTENT, lq.SCHED_STREAMK
 SHAPES = [
-    # M, N, K, block_t, split_k, grid   (0 = automatic; grid > 0 = stream-K)
-    (16, 256, 512, 0, 0, 0),        # the tiny workload
-    (1, 256, 512, 0, 0, 0),
-    (1, 16, 128, 0, 0, 0),          # one K-block, N smaller than a tile
-    (3, 272, 384, 16, 0, 0),        # ragged N (one full + one 16-row tile)
-    (17, 384, 1024, 32, 0, 0),      # ragged M
-    (16, 256, 1024, 16, 1, 0),      # one CTA per tile: direct epilogue
-    (16, 256, 1024, 16, 2, 0),      # cluster split-K, DSMEM reduction
-    (5, 256, 1024, 16, 4, 0),
-    (16, 512, 2048, 16, 8, 0),
-    (32, 256, 1152, 32, 8, 0),      # 9 K-blocks over 8 CTAs: uneven slices
-    (40, 384, 1024, 64, 4, 0),
-    (100, 256, 640, 128, 2, 0),
-    (16, 256, 1024, 16, 0, 2),      # stream-K, one CTA per tile
-    (16, 256, 1024, 16, 0, 3),      # stream-K: split tiles through the workspace
-    (16, 256, 1024, 16, 0, 16),     # one K-block per CTA
-    (64, 512, 512, 64, 0, 7),
-    (100, 256, 640, 128, 0, 5),
-    (128, 384, 256, 128, 0, 0),
-    (300, 256, 512, 256, 0, 0),     # ragged M with 256-token tiles
-    (300, 256, 512, 256, 0, 4),
-    (256, 128, 2048, 256, 0, 9),
+    # M, N, K, block_t, schedule, split_k, grid   (0 / None = automatic)
+    (16, 256, 512, 0, None, 0, 0),        # the tiny workload
+    (1, 256, 512, 0, None, 0, 0),
+    (1, 16, 128, 0, None, 0, 0),          # one K-block, N smaller than a tile
+    (3, 272, 384, 16, T, 0, 0),           # ragged N (one full + one 16-row tile)
+    (17, 384, 1024, 32, T, 0, 0),         # ragged M
+    (16, 256, 1024, 16, T, 1, 0),         # one CTA per tile: direct epilogue
+    (16, 256, 1024, 16, T, 2, 0),         # cluster split-K, DSMEM reduction
+    (5, 256, 1024, 16, T, 4, 0),
+    (16, 512, 2048, 16, T, 8, 0),
+    (32, 256, 1152, 32, T, 8, 0),         # 9 K-blocks over 8 CTAs: uneven slices
+    (40, 384, 1024, 64, T, 4, 0),
+    (100, 256, 640, 128, T, 2, 0),
+    (128, 384, 256, 128, T, 0, 0),
+    (300, 256, 512, 256, T, 0, 0),        # ragged M with 256-token tiles
+    (128, 128, 128, 0, P, 0, 0),          # persistent: one tile
+    (300, 256, 512, 0, P, 0, 0),          # persistent: ragged M, one tile per CTA
+    (256, 384, 1024, 0, P, 0, 2),         # persistent: 3 tiles per CTA, both accumulators reused
+    (1000, 512, 640, 0, P, 0, 3),         # persistent: 32 tiles over 3 CTAs, ragged M
+    (16, 256, 1024, 16, SK, 0, 2),        # stream-K, one CTA per tile
+    (16, 256, 1024, 16, SK, 0, 3),        # stream-K: split tiles through the workspace
+    (16, 256, 1024, 16, SK, 0, 16),       # one K-block per CTA
+    (64, 512, 512, 64, SK, 0, 7),
+    (100, 256, 640, 128, SK, 0, 5),
+    (300, 256, 512, 256, SK, 0, 4),
+    (256, 128, 2048, 256, SK, 0, 9),
 ]
 
 
-@pytest.mark.parametrize("M,N,K,bt,split,grid", SHAPES)
-def test_gemm_parity(M, N, K, bt, split, grid):
+@pytest.mark.parametrize("M,N,K,bt,sched,split,grid", SHAPES)
+def test_gemm_parity(M, N, K, bt, sched, split, grid):
     X, W = synth.make_problem(M, N, K, seed=M * 7 + N + K, n_outliers=2)
     g, o = quantize_both(X, W)
     assert_quant_equal(g, o)
     g_qw, g_s, g_a, g_sc, g_xq, g_sx = g
     o_out, o_acc = oracle.w4a8_gemm(*[o[i] for i in (4, 5, 0, 1, 2, 3)])
-    acc = lq.lq_w4a8_gemm_i32(g_xq, g_qw, g_s, g_a, block_t=bt, split_k=split, grid=grid)
-    out = lq.lq_w4a8_gemm(g_xq, g_sx, g_qw, g_s, g_a, g_sc, block_t=bt, split_k=split, grid=grid)
+    kw = dict(block_t=bt, schedule=sched, split_k=split, grid=grid)
+    acc = lq.lq_w4a8_gemm_i32(g_xq, g_qw, g_s, g_a, **kw)
+    out = lq.lq_w4a8_gemm(g_xq, g_sx, g_qw, g_s, g_a, g_sc, **kw)
     assert lq.lq_get_device_error() == 0
     np.testing.assert_array_equal(_np(acc), o_acc)
     ulps = _bf16_ulps(_u16(out), o_out)
     assert ulps.max() <= 1
     # a second call on the same (restored) workspace gives the same result
-    out2 = lq.lq_w4a8_gemm(g_xq, g_sx, g_qw, g_s, g_a, g_sc, block_t=bt, split_k=split, grid=grid)
-    acc2 = lq.lq_w4a8_gemm_i32(g_xq, g_qw, g_s, g_a, block_t=bt, split_k=split, grid=grid)
+    out2 = lq.lq_w4a8_gemm(g_xq, g_sx, g_qw, g_s, g_a, g_sc, **kw)
+    acc2 = lq.lq_w4a8_gemm_i32(g_xq, g_qw, g_s, g_a, **kw)
     torch.cuda.synchronize()
     assert torch.equal(out, out2) and torch.equal(acc, acc2)
 
@@ -155,7 +161,7 @@ def test_workspace_left_zero():
     X, W = synth.make_problem(M, N, K, seed=3)
     qw, s, a, sc = lq.lq_quantize_weights(W.to(DEV))
     xq, sx = lq.lq_quantize_act(X.to(DEV))
-    need = lq.lq_w4a8_gemm_workspace_size(M, N, K, 16, 0, 5)
+    need = lq.lq_w4a8_gemm_workspace_size(M, N, K, 16, 0, 5, lq.SCHED_STREAMK)
     assert need > 0
     ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     for _ in range(3):

@@ -26,6 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblq_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lq.h")
 GROUP = 64
+SCHED_AUTO, SCHED_TILES, SCHED_PERSISTENT, SCHED_STREAMK = 0, 1, 2, 3
 
 STATUS = {
     0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED_SHAPE", 3: "LQ_ERR_MISALIGNED",
@@ -62,9 +63,9 @@ def load_library(path: str = LIB_PATH):
             "lq_quantize_weights": ([P, I, I, I, P, P, P, P, P], I),
             "lq_quantize_act": ([P, I, I, P, P, P], I),
             "lq_w4a8_gemm_workspace_size": ([I, I, I], Z),
-            "lq_w4a8_gemm_workspace_size_ex": ([I, I, I, I, I, I], Z),
+            "lq_w4a8_gemm_workspace_size_ex": ([I, I, I, I, I, I, I], Z),
             "lq_w4a8_gemm": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, P], I),
-            "lq_w4a8_gemm_ex": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, I, I, I, I, P], I),
+            "lq_w4a8_gemm_ex": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, I, I, I, I, I, P], I),
             "lq_w4a8_gemm_i32": ([P, P, P, P, P, I, I, I, I, P, Z, P], I),
             "lq_dequant_weights_i8": ([P, P, P, I, I, I, P, P], I),
             "lq_get_device_error": ([P], I),
@@ -167,15 +168,27 @@ def lq_quantize_act(X: torch.Tensor, out=None):
     return xq, sx
 
 
+def _sched(schedule, split_k, grid):
+    """Default the schedule from the other knobs (split_k -> tiles, grid -> stream-K)."""
+    if schedule is not None:
+        return schedule
+    if grid:
+        return SCHED_STREAMK
+    if split_k:
+        return SCHED_TILES
+    return SCHED_AUTO
+
+
 def lq_w4a8_gemm_workspace_size(M: int, N: int, K: int, block_t: int = 0, split_k: int = 0,
-                                grid: int = 0) -> int:
+                                grid: int = 0, schedule: int | None = None) -> int:
     lib = load_library()
-    if block_t == 0 and split_k == 0 and grid == 0:
+    sch = _sched(schedule, split_k, grid)
+    if block_t == 0 and split_k == 0 and grid == 0 and sch == SCHED_AUTO:
         return int(lib.lq_w4a8_gemm_workspace_size(M, N, K))
-    return int(lib.lq_w4a8_gemm_workspace_size_ex(M, N, K, block_t, split_k, grid))
+    return int(lib.lq_w4a8_gemm_workspace_size_ex(M, N, K, block_t, sch, split_k, grid))
 
 
-def _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, split_k, grid, out_i32, ws):
+def _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, split_k, grid, out_i32, ws, schedule=None):
     lib = load_library()
     _need(x_q, torch.int8, "x_q")
     M, K = x_q.shape
@@ -191,29 +204,33 @@ def _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, split_k, grid, out
         out = torch.empty(M, N, dtype=odt, device=x_q.device)
     _need(out, odt, "out", (M, N))
     with torch.cuda.device(x_q.device):
-        need = lq_w4a8_gemm_workspace_size(M, N, K, block_t, split_k, grid)
+        sch = _sched(schedule, split_k, grid)
+        need = lq_w4a8_gemm_workspace_size(M, N, K, block_t, split_k, grid, sch)
         if ws is None:
             ws = workspace(need, x_q.device)
         nbytes = ws.numel() * ws.element_size() if ws is not None else 0
         _check("lq_w4a8_gemm", lib.lq_w4a8_gemm_ex(
             _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out),
-            M, N, K, group, _ptr(ws), nbytes, block_t, split_k, grid, 1 if out_i32 else 0,
+            M, N, K, group, _ptr(ws), nbytes, block_t, sch, split_k, grid, 1 if out_i32 else 0,
             _stream(x_q.device)))
     return out
 
 
 def lq_w4a8_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP,
-                 block_t: int = 0, split_k: int = 0, grid: int = 0, workspace_buf=None):
+                 block_t: int = 0, split_k: int = 0, grid: int = 0, workspace_buf=None,
+                 schedule: int | None = None):
     """W4A8 GEMM: bf16(float(x_q @ dequant(qw)^T) * s_x[m] * s_c[n]) -> [M, N] bf16.
 
-    block_t / split_k / grid override the automatic schedule (see lq_w4a8_gemm_ex in lq.h)."""
-    return _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, split_k, grid, False, workspace_buf)
+    block_t / schedule / split_k / grid override the automatic schedule (lq_w4a8_gemm_ex in lq.h)."""
+    return _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, split_k, grid, False, workspace_buf,
+                 schedule)
 
 
 def lq_w4a8_gemm_i32(x_q, qw, s_u8, a_u8, out=None, group: int = GROUP, block_t: int = 0,
-                     split_k: int = 0, grid: int = 0, workspace_buf=None):
+                     split_k: int = 0, grid: int = 0, workspace_buf=None, schedule: int | None = None):
     """The int32 accumulators x_q @ dequant(qw)^T -> [M, N] int32."""
-    return _gemm(x_q, None, qw, s_u8, a_u8, None, out, group, block_t, split_k, grid, True, workspace_buf)
+    return _gemm(x_q, None, qw, s_u8, a_u8, None, out, group, block_t, split_k, grid, True, workspace_buf,
+                 schedule)
 
 
 def lq_dequant_weights_i8(qw, s_u8, a_u8, group: int = GROUP, out=None):

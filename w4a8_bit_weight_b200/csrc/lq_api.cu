@@ -13,6 +13,7 @@
 #include "../../include/lq.h"
 #include "lq_device.cuh"
 #include "lq_gemm_kernel.cuh"
+#include "lq_gemm_persistent.cuh"
 #include "lq_quant_kernels.cuh"
 
 namespace {
@@ -83,7 +84,10 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
 }
 
 // ------------------------------------------------------------- schedule
+enum SchedKind { kSchedAuto = 0, kSchedTiles = 1, kSchedPersistent = 2, kSchedStreamK = 3 };
+
 struct Schedule {
+  int kind = kSchedTiles;
   int bt = 0;        // tokens per tile
   int cs = 1;        // CTAs per tile in a cluster (split-K), 0 = stream-K
   int tiles_m = 0, tiles_n = 0, KB = 0;
@@ -115,18 +119,41 @@ bool pdl_enabled() {
   return on;
 }
 
-// split_k > 0: cluster split of that many CTAs per tile; grid > 0: stream-K
-// over that many CTAs; both 0: automatic.
-Schedule make_schedule(int M, int N, int K, int block_t, int split_k, int grid, int sms) {
+bool valid_schedule(int M, int block_t, int schedule, int split_k, int grid) {
+  if (block_t != 0 && !valid_block_t(block_t)) return false;
+  if (split_k < 0 || grid < 0) return false;
+  switch (schedule) {
+    case kSchedAuto:
+      return split_k == 0 && grid == 0;
+    case kSchedTiles:
+      return grid == 0 && (split_k == 0 || valid_split(block_t ? block_t : auto_block_t(M > 0 ? M : 1), split_k));
+    case kSchedPersistent:
+      return split_k == 0 && (block_t == 0 || block_t == lq::kPBT);
+    case kSchedStreamK:
+      return split_k == 0;
+  }
+  return false;
+}
+
+Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms) {
   Schedule s;
-  s.bt = block_t ? block_t : auto_block_t(M);
+  int kind = schedule;
+  int bt = block_t ? block_t : auto_block_t(M);
+  if (kind == kSchedAuto) {
+    // many tiles of 128 tokens: persistent; otherwise one cluster per tile
+    const long long t128 = (long long)((M + lq::kPBT - 1) / lq::kPBT) * ((N + lq::kBlockN - 1) / lq::kBlockN);
+    kind = (bt == lq::kPBT && t128 >= sms) ? kSchedPersistent : kSchedTiles;
+  }
+  if (kind == kSchedPersistent) bt = lq::kPBT;
+  s.kind = kind;
+  s.bt = bt;
   s.tiles_m = (M + s.bt - 1) / s.bt;
   s.tiles_n = (N + lq::kBlockN - 1) / lq::kBlockN;
   s.KB = K / lq::kBlockK;
   s.tiles = (long long)s.tiles_m * s.tiles_n;
   s.U = s.tiles * s.KB;
-  if (grid > 0) {
-    long long g = grid;
+  if (kind == kSchedStreamK) {
+    long long g = grid > 0 ? grid : sms;
     if (g > s.U) g = s.U;
     if (g > INT_MAX) g = INT_MAX;
     s.cs = 0;
@@ -140,6 +167,13 @@ Schedule make_schedule(int M, int N, int K, int block_t, int split_k, int grid, 
       const size_t acc = (size_t)s.tiles * s.bt * lq::kBlockN * sizeof(int32_t);
       s.ws_bytes = acc + (((size_t)s.tiles * sizeof(unsigned) + 15) / 16) * 16;
     }
+    return s;
+  }
+  if (kind == kSchedPersistent) {
+    long long g = grid > 0 ? grid : sms;
+    if (g > s.tiles) g = s.tiles;
+    s.cs = 1;
+    s.grid = (int)g;
     return s;
   }
   int cs = split_k;
@@ -227,6 +261,12 @@ lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const CUtenso
 template <bool I32>
 lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
                       const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  if (s.kind == kSchedPersistent) {
+    auto kern = lq::w4a8_gemm_persistent_kernel<I32>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::kPSmemBytes) != cudaSuccess)
+      return LQ_ERR_CUDA;
+    return launch_ex(kern, s.grid, lq::kPThreads, lq::kPSmemBytes, 1, pdl_enabled(), st, tx, tw, ts, ta, a);
+  }
   switch (s.bt) {
     case 16: return launch_gemm_bt<16, I32>(s, tx, tw, ts, ta, a, st);
     case 32: return launch_gemm_bt<32, I32>(s, tx, tw, ts, ta, a, st);
@@ -239,14 +279,11 @@ lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMa
 
 lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                     const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
-                    void* workspace, size_t ws_bytes, int block_t, int split_k, int grid, bool out_i32,
-                    void* stream) {
+                    void* workspace, size_t ws_bytes, int block_t, int schedule, int split_k, int grid,
+                    bool out_i32, void* stream) {
   lq_status st = check_gemm_shape(M, N, K, group);
   if (st != LQ_OK) return st;
-  if (block_t != 0 && !valid_block_t(block_t)) return LQ_ERR_INVALID_ARG;
-  if (grid < 0 || split_k < 0 || (grid > 0 && split_k > 0)) return LQ_ERR_INVALID_ARG;
-  if (split_k > 0 && !valid_split(block_t ? block_t : auto_block_t(M > 0 ? M : 1), split_k))
-    return LQ_ERR_INVALID_ARG;
+  if (!valid_schedule(M, block_t, schedule, split_k, grid)) return LQ_ERR_INVALID_ARG;
   if (M == 0) return LQ_OK;
   if (!x_q || !qw || !s_u8 || !a_u8 || !out || (!out_i32 && (!s_x || !s_c))) return LQ_ERR_INVALID_ARG;
   if (!aligned(x_q, 16) || !aligned(qw, 16) || !aligned(s_u8, 16) || !aligned(a_u8, 16) ||
@@ -255,7 +292,7 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
-  const Schedule s = make_schedule(M, N, K, block_t, split_k, grid, dev->sms);
+  const Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms);
   if (s.split) {
     if (!workspace || ws_bytes < s.ws_bytes) return LQ_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return LQ_ERR_MISALIGNED;
@@ -335,40 +372,39 @@ lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, float* 
                    static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(X_bf16), K, x_q, s_x);
 }
 
-size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int split_k, int grid) {
+size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int schedule, int split_k, int grid) {
   if (check_gemm_shape(M, N, K, LQ_GROUP) != LQ_OK || M == 0) return 0;
-  if (block_t != 0 && !valid_block_t(block_t)) return 0;
-  if (grid < 0 || split_k < 0) return 0;
+  if (!valid_schedule(M, block_t, schedule, split_k, grid)) return 0;
   DeviceInfo* dev = nullptr;
   int sms = 148;
   if (current_device(&dev) == LQ_OK) sms = dev->sms;
-  return make_schedule(M, N, K, block_t, split_k, grid, sms).ws_bytes;
+  return make_schedule(M, N, K, block_t, schedule, split_k, grid, sms).ws_bytes;
 }
 
 size_t lq_w4a8_gemm_workspace_size(int M, int N, int K) {
-  return lq_w4a8_gemm_workspace_size_ex(M, N, K, 0, 0, 0);
+  return lq_w4a8_gemm_workspace_size_ex(M, N, K, 0, 0, 0, 0);
 }
 
 lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                           const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
-                          void* workspace, size_t workspace_bytes, int block_t, int split_k, int grid,
-                          int out_i32, void* stream) {
+                          void* workspace, size_t workspace_bytes, int block_t, int schedule, int split_k,
+                          int grid, int out_i32, void* stream) {
   return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out, M, N, K, group, workspace, workspace_bytes, block_t,
-                   split_k, grid, out_i32 != 0, stream);
+                   schedule, split_k, grid, out_i32 != 0, stream);
 }
 
 lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                        const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K, int group,
                        void* workspace, size_t workspace_bytes, void* stream) {
   return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes, 0, 0,
-                   0, false, stream);
+                   0, 0, false, stream);
 }
 
 lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8,
                            int32_t* acc, int M, int N, int K, int group, void* workspace,
                            size_t workspace_bytes, void* stream) {
   return gemm_impl(x_q, nullptr, qw, s_u8, a_u8, nullptr, acc, M, N, K, group, workspace, workspace_bytes, 0,
-                   0, 0, true, stream);
+                   0, 0, 0, true, stream);
 }
 
 lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8, int N, int K,
