@@ -141,6 +141,7 @@ LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t
 #define LQ_SCHED_TILES 1      /* one cluster of split_k CTAs per tile */
 #define LQ_SCHED_PERSISTENT 2 /* grid CTAs loop over 128-token tiles */
 #define LQ_SCHED_STREAMK 3    /* grid CTAs share the K-blocks of all tiles */
+#define LQ_SCHED_PAIR 4       /* CTA pairs (tcgen05 cta_group::2) loop over 256 x 256 tiles */
 
 /*
  * lq_w4a8_gemm_ex -- lq_w4a8_gemm with the schedule chosen by the caller
@@ -157,6 +158,11 @@ LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t
  *             LQ_SCHED_PERSISTENT: grid CTAs (0 = one per SM) loop over the
  *               tiles, overlapping each tile's epilogue with the next tile's
  *               main loop.  split_k must be 0.
+ *             LQ_SCHED_PAIR: grid/2 clusters of two CTAs (0 = one CTA per SM)
+ *               loop over tiles of 256 weight rows x 256 tokens; each MMA
+ *               instruction spans both SMs of a pair.  Requires K % 256 == 0
+ *               (else LQ_ERR_UNSUPPORTED_SHAPE); block_t must be 0 or 256;
+ *               split_k must be 0.
  *             LQ_SCHED_STREAMK: the K-blocks of all tiles are spread evenly
  *               over grid CTAs (0 = one per SM; clamped to the number of
  *               K-blocks of work); tiles shared by several CTAs are reduced

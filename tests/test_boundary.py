@@ -48,7 +48,7 @@ def gemm(lib, M=16, N=256, K=512, group=64, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=
     (dict(sx=P(0)), 1), (dict(sc=P(0)), 1),
     (dict(x=ODD), 3), (dict(qw=ODD), 3), (dict(s=ODD), 3), (dict(a=ODD), 3), (dict(out=ODD), 3),
     (dict(sx=P((1 << 20) + 2)), 3),
-    (dict(bt=48), 1), (dict(sched=4), 1), (dict(sched=-1), 1),
+    (dict(bt=48), 1), (dict(sched=6), 1), (dict(sched=-1), 1),
     (dict(sched=3, grid=-1), 1), (dict(sched=1, split=-1), 1), (dict(sched=1, split=3), 1),
     (dict(split=2), 1), (dict(grid=4), 1),        # the automatic schedule takes no split or grid
     (dict(sched=1, split=2, grid=4), 1),          # a cluster split has no grid
@@ -56,6 +56,9 @@ def gemm(lib, M=16, N=256, K=512, group=64, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=
     (dict(sched=1, bt=64, split=8), 1),           # split 8 only for tiles of <= 32 tokens
     (dict(sched=1, bt=256, split=2), 1),          # 256-token tiles are never split
     (dict(sched=2, bt=64), 1),                    # the persistent schedule uses 128-token tiles
+    (dict(sched=4, bt=128), 1),                   # CTA pairs use 256-token tiles
+    (dict(sched=4, split=2), 1),
+    (dict(sched=5), 1),
 ])
 def test_gemm_rejects_before_launch(lib, kw, code):
     assert gemm(lib, **kw) == code

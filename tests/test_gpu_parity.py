@@ -104,7 +104,7 @@ def test_dequant_identity_all_codes_on_gpu():
 # GEMM: int32 bit-exact and bf16 within 1 ulp, across schedules
 # ----------------------------------------------------------------------------
 
-T, P, SK = lq.SCHED_TILES, lq.SCHED_PERSISTENT, lq.SCHED_STREAMK
+T, P, SK, PR = lq.SCHED_TILES, lq.SCHED_PERSISTENT, lq.SCHED_STREAMK, lq.SCHED_PAIR
 SHAPES = [
     # M, N, K, block_t, schedule, split_k, grid   (0 / None = automatic)
     (16, 256, 512, 0, None, 0, 0),        # the tiny workload
@@ -125,6 +125,10 @@ SHAPES = [
     (300, 256, 512, 0, P, 0, 0),          # persistent: ragged M, one tile per CTA
     (256, 384, 1024, 0, P, 0, 2),         # persistent: 3 tiles per CTA, both accumulators reused
     (1000, 512, 640, 0, P, 0, 3),         # persistent: 32 tiles over 3 CTAs, ragged M
+    (256, 256, 512, 0, PR, 0, 0),         # CTA pair: one 256 x 256 tile
+    (300, 272, 1024, 0, PR, 0, 0),        # CTA pairs: ragged M and N
+    (512, 512, 2048, 0, PR, 0, 2),        # one pair, four tiles: accumulator handed back and forth
+    (1000, 768, 768, 0, PR, 0, 4),        # two pairs, 12 tiles, ragged M
     (16, 256, 1024, 16, SK, 0, 2),        # stream-K, one CTA per tile
     (16, 256, 1024, 16, SK, 0, 3),        # stream-K: split tiles through the workspace
     (16, 256, 1024, 16, SK, 0, 16),       # one K-block per CTA

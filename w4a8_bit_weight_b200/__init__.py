@@ -26,7 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblq_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lq.h")
 GROUP = 64
-SCHED_AUTO, SCHED_TILES, SCHED_PERSISTENT, SCHED_STREAMK = 0, 1, 2, 3
+SCHED_AUTO, SCHED_TILES, SCHED_PERSISTENT, SCHED_STREAMK, SCHED_PAIR = 0, 1, 2, 3, 4
 
 STATUS = {
     0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED_SHAPE", 3: "LQ_ERR_MISALIGNED",

@@ -14,6 +14,7 @@
 #include "lq_device.cuh"
 #include "lq_gemm_kernel.cuh"
 #include "lq_gemm_persistent.cuh"
+#include "lq_gemm_pair.cuh"
 #include "lq_quant_kernels.cuh"
 
 namespace {
@@ -84,7 +85,7 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
 }
 
 // ------------------------------------------------------------- schedule
-enum SchedKind { kSchedAuto = 0, kSchedTiles = 1, kSchedPersistent = 2, kSchedStreamK = 3 };
+enum SchedKind { kSchedAuto = 0, kSchedTiles = 1, kSchedPersistent = 2, kSchedStreamK = 3, kSchedPair = 4 };
 
 struct Schedule {
   int kind = kSchedTiles;
@@ -131,6 +132,8 @@ bool valid_schedule(int M, int block_t, int schedule, int split_k, int grid) {
       return split_k == 0 && (block_t == 0 || block_t == lq::kPBT);
     case kSchedStreamK:
       return split_k == 0;
+    case kSchedPair:
+      return split_k == 0 && (block_t == 0 || block_t == lq::kQBT);
   }
   return false;
 }
@@ -140,9 +143,29 @@ Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split
   int kind = schedule;
   int bt = block_t ? block_t : auto_block_t(M);
   if (kind == kSchedAuto) {
-    // many tiles of 128 tokens: persistent; otherwise one cluster per tile
+    // enough 256 x 256 tiles to give every CTA pair one: CTA pairs; many tiles
+    // of 128 tokens: persistent; otherwise one cluster per tile
     const long long t128 = (long long)((M + lq::kPBT - 1) / lq::kPBT) * ((N + lq::kBlockN - 1) / lq::kBlockN);
-    kind = (bt == lq::kPBT && t128 >= sms) ? kSchedPersistent : kSchedTiles;
+    const long long t256 = (long long)((M + lq::kQBT - 1) / lq::kQBT) * ((N + lq::kQBN - 1) / lq::kQBN);
+    if (block_t == 0 && K % lq::kQBK == 0 && t256 >= sms / 2)
+      kind = kSchedPair;
+    else
+      kind = (bt == lq::kPBT && t128 >= sms) ? kSchedPersistent : kSchedTiles;
+  }
+  if (kind == kSchedPair) {
+    s.kind = kind;
+    s.bt = lq::kQBT;
+    s.tiles_m = (M + lq::kQBT - 1) / lq::kQBT;
+    s.tiles_n = (N + lq::kQBN - 1) / lq::kQBN;
+    s.KB = K / lq::kBlockK;
+    s.tiles = (long long)s.tiles_m * s.tiles_n;
+    s.U = s.tiles;  // the pair kernel takes the tile count here
+    long long pairs = grid > 0 ? (grid + 1) / 2 : sms / 2;
+    if (pairs > s.tiles) pairs = s.tiles;
+    if (pairs < 1) pairs = 1;
+    s.cs = 2;
+    s.grid = (int)(2 * pairs);
+    return s;
   }
   if (kind == kSchedPersistent) bt = lq::kPBT;
   s.kind = kind;
@@ -190,6 +213,11 @@ Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split
   s.cs = cs;
   s.grid = (int)(s.tiles * cs);
   return s;
+}
+
+lq_status check_schedule_shape(const Schedule& s, int K) {
+  if (s.kind == kSchedPair && K % lq::kQBK != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return LQ_OK;
 }
 
 lq_status check_gemm_shape(int M, int N, int K, int group) {
@@ -261,6 +289,12 @@ lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const CUtenso
 template <bool I32>
 lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
                       const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  if (s.kind == kSchedPair) {
+    auto kern = lq::w4a8_gemm_pair_kernel<I32>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::kQSmemBytes) != cudaSuccess)
+      return LQ_ERR_CUDA;
+    return launch_ex(kern, s.grid, lq::kQThreads, lq::kQSmemBytes, 2, pdl_enabled(), st, tx, tw, ts, ta, a);
+  }
   if (s.kind == kSchedPersistent) {
     auto kern = lq::w4a8_gemm_persistent_kernel<I32>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::kPSmemBytes) != cudaSuccess)
@@ -293,18 +327,25 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   st = current_device(&dev);
   if (st != LQ_OK) return st;
   const Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms);
+  st = check_schedule_shape(s, K);
+  if (st != LQ_OK) return st;
   if (s.split) {
     if (!workspace || ws_bytes < s.ws_bytes) return LQ_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return LQ_ERR_MISALIGNED;
   }
   CUtensorMap tx, tw, ts, ta;
-  if (!make_map_u8(&tx, x_q, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, s.bt,
+  // the pair kernel loads 128 tokens and 128 weight rows per CTA with 256 K per stage
+  const bool pair = (s.kind == kSchedPair);
+  const uint32_t x_rows = pair ? 128u : (uint32_t)s.bt;
+  const uint32_t w_box = pair ? (uint32_t)lq::kQBK / 2 : (uint32_t)lq::kBlockK / 2;
+  const uint32_t sa_groups = pair ? (uint32_t)lq::kQBK / LQ_GROUP : 2u;
+  if (!make_map_u8(&tx, x_q, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, x_rows,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, lq::kBlockK / 2, lq::kBlockN,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_u8(&ts, s_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, 2,
+      !make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, w_box, lq::kBlockN,
+                   pair ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_u8(&ts, s_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, sa_groups,
                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_u8(&ta, a_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, 2,
+      !make_map_u8(&ta, a_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, sa_groups,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return LQ_ERR_CUDA;
   lq::GemmArgs a;

@@ -1,0 +1,379 @@
+// lq_gemm_pair.cuh -- W4A8 GEMM on CTA pairs (tcgen05 cta_group::2) for
+// large token counts.
+//
+// A cluster of two CTAs on two SMs computes one tile of 256 weight rows x 256
+// tokens with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32 per
+// instruction):
+//   * each CTA expands ITS 128 weight rows into ITS tensor memory (the MMA's
+//     A operand, one TMEM lane per row, as in the one-CTA kernels);
+//   * each CTA loads HALF of the tokens (128) into its shared memory (the
+//     MMA's B operand is split by N across the pair), so every activation
+//     byte fetched serves 256 weight rows;
+//   * each CTA's TMEM holds the int32 accumulators of its 128 weight rows for
+//     all 256 tokens;
+//   * one thread of the even CTA issues every MMA for both SMs: 128 cycles of
+//     tensor work per SM per instruction, enough to hide the issue cost.
+// Stages carry 256 K (four groups of 64).  The accumulator is single: the
+// epilogue warps of both CTAs hand it back as soon as their last TMEM load
+// has landed, so only the loads (not the stores) sit between two tiles.
+//
+// Hand-offs between the two CTAs:
+//   expansion done  -> arrive on the even CTA's afull[stage] (remote for odd)
+//   stage consumed  -> tcgen05.commit multicast to empty[stage] of both CTAs
+//   tile finished   -> tcgen05.commit multicast to accfull of both CTAs
+//   accum. loaded   -> arrive on the even CTA's accempty (remote for odd)
+// No TMA load uses cluster multicast: each CTA loads its own data.
+//
+// Warp roles (576 threads):
+//   warp 0        TMA producer
+//   warp 1        TMEM allocation (both CTAs); MMA issue (even CTA)
+//   warps 2-9     expansion: two groups of four warps, alternate stages
+//   warps 10-17   epilogue: two warps per TMEM lane quarter, 128 tokens each
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "lq_device.cuh"
+#include "lq_gemm_kernel.cuh"
+
+namespace lq {
+
+constexpr int kQBT = 256;                     // tokens per tile (MMA N)
+constexpr int kQBN = 256;                     // weight rows per tile (MMA M, 128 per CTA)
+constexpr int kQBK = 256;                     // K per stage
+constexpr int kQStages = 4;
+constexpr int kQExpGroups = 2;
+constexpr int kQEpiWarp0 = 2 + 4 * kQExpGroups;
+constexpr int kQThreads = 32 * (kQEpiWarp0 + 8);
+constexpr int kQXSub = 128 * 128;             // one 128-token x 128-K SW128 sub-tile
+constexpr int kQXBytes = 2 * kQXSub;          // 32 KB: this CTA's 128 tokens x 256 K
+constexpr int kQWBytes = 128 * kQBK / 2;      // 16 KB: 128 rows x 256 codes, 128-byte rows
+constexpr int kQSABytes = (kQBK / 64) * 128;  // 4 groups x 128 rows
+constexpr int kQStageBytes = round_up_c(kQXBytes + kQWBytes + 2 * kQSABytes, 1024);
+constexpr uint32_t kQTx = kQXBytes + kQWBytes + 2 * kQSABytes;
+constexpr int kQAccCols = kQBT;               // one accumulator
+constexpr int kQSlotCols = kQBK / 4;          // 64 TMEM columns per expanded stage
+constexpr int kQBarBytes = 256;
+constexpr int kQSmemBytes = kQStages * kQStageBytes + kQBarBytes + 1024;
+static_assert(kQAccCols + kQStages * kQSlotCols <= 512, "TMEM budget");
+static_assert(kQSmemBytes <= 232448, "shared memory budget");
+static_assert(kQStages % kQExpGroups == 0, "stages per expansion group");
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[256 x N] (+)= A[256 x 32] * B[N x 32]^T over the CTA pair (int8 -> int32).
+__device__ __forceinline__ void mma_i8_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives on the mbarrier at this shared-memory offset in every CTA of
+// `cta_mask` once all prior tcgen05 operations of the pair have completed.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t idesc_i8_pair() {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kQBT >> 3) << 17) | (uint32_t(kQBN >> 4) << 24);
+}
+
+// Arrive on the even CTA's copy of `bar` (local arrive on the even CTA).
+__device__ __forceinline__ void arrive_on_leader(uint64_t* bar, uint32_t crank) {
+  if (crank == 0)
+    mbar_arrive(bar);
+  else
+    mbar_arrive_remote(mapa_shared(smem_u32(bar), 0));
+}
+
+// One elected lane waits; the decision is shared with the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, bool cluster) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = cluster ? mbar_wait_cluster(bar, parity, abort_flag) : mbar_wait(bar, parity, abort_flag);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+template <bool OUT_I32>
+__global__ void __launch_bounds__(kQThreads, 1)
+    w4a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                          const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
+                          const GemmArgs p) {
+  constexpr int S = kQStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kQStageBytes);
+  uint64_t* afull = full + S;
+  uint64_t* empty = afull + S;
+  uint64_t* accfull = empty + S;
+  uint64_t* accempty = accfull + 1;
+  uint64_t* drain = accempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool leader = (lane == 0);
+  const uint32_t crank = cluster_ctarank();
+  const bool even = (crank == 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], 8);   // four expansion warps of each CTA
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accempty, 16);     // eight epilogue warps of each CTA
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_s);
+    tma_prefetch_desc(&tm_a);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // both CTAs' barriers exist before any remote arrive or multicast commit
+  cluster_arrive();
+  cluster_wait();
+
+  const int KS = p.K / kQBK;                 // stages per tile
+  const int tiles_m = p.tiles_m;
+  const int tiles = (int)(p.U);             // host passes the tile count in U
+  const int cid = blockIdx.x >> 1;
+  const int ncl = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint64_t pol_stream = 0, pol_keep = 0;
+    if (leader) {
+      pol_stream = l2_policy_evict_first();
+      pol_keep = l2_policy_evict_last();
+    }
+    const int P = cid < tiles ? min(S, KS) : 0;
+    const int t0n = cid / tiles_m, t0m = cid % tiles_m;
+    if (leader)
+      for (int i = 0; i < P; ++i) {
+        uint8_t* sb = smem + i * kQStageBytes;
+        mbar_arrive_expect_tx(&full[i], kQTx);
+        tma_load_2d(sb + kQXBytes, &tm_w, &full[i], i * (kQBK / 2), t0n * kQBN + (int)crank * 128, pol_stream);
+        tma_load_2d(sb + kQXBytes + kQWBytes, &tm_s, &full[i], t0n * kQBN + (int)crank * 128, i * 4, pol_stream);
+        tma_load_2d(sb + kQXBytes + kQWBytes + kQSABytes, &tm_a, &full[i], t0n * kQBN + (int)crank * 128, i * 4,
+                    pol_stream);
+      }
+    griddep_wait();
+    if (leader)
+      for (int i = 0; i < P; ++i) {
+        uint8_t* sb = smem + i * kQStageBytes;
+        tma_load_2d(sb, &tm_x, &full[i], i * kQBK, t0m * kQBT + (int)crank * 128, pol_keep);
+        tma_load_2d(sb + kQXSub, &tm_x, &full[i], i * kQBK + 128, t0m * kQBT + (int)crank * 128, pol_keep);
+      }
+    __syncwarp();
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = (1u << P) - 1u, issued_par = 0;
+    int it = 0;
+    for (int tile = cid; tile < tiles; tile += ncl) {
+      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      const int xrow = tm * kQBT + (int)crank * 128;
+      const int wrow = tn * kQBN + (int)crank * 128;
+      for (int kb = 0; kb < KS; ++kb, ++it) {
+        if (it >= P) {
+          if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, false)) goto producer_done;
+          if (leader) {
+            uint8_t* sb = smem + stage * kQStageBytes;
+            mbar_arrive_expect_tx(&full[stage], kQTx);
+            tma_load_2d(sb, &tm_x, &full[stage], kb * kQBK, xrow, pol_keep);
+            tma_load_2d(sb + kQXSub, &tm_x, &full[stage], kb * kQBK + 128, xrow, pol_keep);
+            tma_load_2d(sb + kQXBytes, &tm_w, &full[stage], kb * (kQBK / 2), wrow, pol_stream);
+            tma_load_2d(sb + kQXBytes + kQWBytes, &tm_s, &full[stage], wrow, kb * 4, pol_stream);
+            tma_load_2d(sb + kQXBytes + kQWBytes + kQSABytes, &tm_a, &full[stage], wrow, kb * 4, pol_stream);
+          }
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  producer_done:
+    if (leader && *abort_flag) {
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) {
+          const uint32_t a = smem_u32(&full[s]);
+          const unsigned long long t0w = globaltimer();
+          while (!mbar_try_wait(a, (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
+          }
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer (even CTA)
+    if (even) {
+      const uint32_t idesc = idesc_i8_pair();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool any = false;
+      int j = 0;
+      for (int tile = cid; tile < tiles; tile += ncl, ++j) {
+        // the single accumulator is free once both CTAs' epilogues have loaded it
+        if (!warp_wait(accempty, ((uint32_t)j & 1u) ^ 1u, abort_flag, true)) goto mma_done;
+        tc_fence_after();
+        for (int kb = 0; kb < KS; ++kb) {
+          if (!warp_wait(&afull[stage], phase, abort_flag, true)) goto mma_done;
+          tc_fence_after();
+          if (leader) {
+            const uint32_t xs = smem_u32(smem + stage * kQStageBytes);
+            const uint32_t a_col = tmem_base + kQAccCols + stage * kQSlotCols;
+#pragma unroll
+            for (int jj = 0; jj < kQBK / 32; ++jj) {
+              const uint64_t bdesc = smem_desc_k_sw128(xs + (jj >> 2) * kQXSub) + (uint64_t)(2 * (jj & 3));
+              mma_i8_ts_pair(tmem_base, a_col + jj * 8, bdesc, idesc, (kb > 0 || jj > 0) ? 1u : 0u);
+            }
+            tc_commit_pair_mc(&empty[stage], 0x3);
+          }
+          __syncwarp();
+          any = true;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (leader) tc_commit_pair_mc(accfull, 0x3);
+        __syncwarp();
+      }
+      griddep_launch_dependents();
+    mma_done:
+      if (leader && any) {
+        tc_commit_pair_mc(drain, 0x1);
+        const uint32_t a = smem_u32(drain);
+        const unsigned long long t0w = globaltimer();
+        while (!mbar_try_wait(a, 0) && globaltimer() - t0w < 100000000ull) {
+        }
+      }
+    }
+  } else if (warp < kQEpiWarp0) {
+    // ------------------------------------------------------ expansion warps
+    const int sub = warp & 3;
+    const int grp = (warp - 2) >> 2;
+    const int r = sub * 32 + lane;
+    const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
+    const int sw = r & 7;                // 128-byte swizzle of this row's 16-byte chunks
+    int ntiles = 0;
+    for (int tile = cid; tile < tiles; tile += ncl) ++ntiles;
+    const int total = ntiles * KS;
+    for (int it = grp; it < total; it += kQExpGroups) {
+      const int stage = it % S;
+      const uint32_t phase = (uint32_t)(it / S) & 1u;
+      if (!warp_wait(&full[stage], phase, abort_flag, false)) goto exp_done;
+      tc_fence_after();
+      const uint8_t* sb = smem + stage * kQStageBytes;
+      const uint8_t* ss = sb + kQXBytes + kQWBytes;
+      const uint32_t wrow = smem_u32(sb + kQXBytes) + r * (kQBK / 2);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {        // 128 K per half: groups 2h, 2h+1
+        const uint32_t s0 = ss[(2 * h) * 128 + r], s1 = ss[(2 * h + 1) * 128 + r];
+        const uint32_t a0 = (uint32_t)ss[kQSABytes + (2 * h) * 128 + r] * 0x01010101u;
+        const uint32_t a1 = (uint32_t)ss[kQSABytes + (2 * h + 1) * 128 + r] * 0x01010101u;
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 q = lds128(wrow + (((4 * h + c) ^ sw) << 4));
+          const uint32_t s = c < 2 ? s0 : s1;
+          const uint32_t a4 = c < 2 ? a0 : a1;
+          lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
+          lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
+          lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
+          lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
+        }
+        tmem_st_32x32b_x32(t_lane + kQAccCols + stage * kQSlotCols + h * 32, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_on_leader(&afull[stage], crank);
+    }
+  exp_done:;
+  } else {
+    // ------------------------------------------------------- epilogue warps
+    const int sub = warp & 3;
+    const int e = (warp - kQEpiWarp0) >> 2;   // tokens [128e, 128e + 128) of the tile
+    const int r = sub * 32 + lane;
+    const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
+    griddep_wait();
+    int j = 0;
+    for (int tile = cid; tile < tiles; tile += ncl, ++j) {
+      if (!warp_wait(accfull, (uint32_t)j & 1u, abort_flag, false)) goto epi_done;
+      tc_fence_after();
+      const int tm = tile % tiles_m, tn = tile / tiles_m;
+      const int n = tn * kQBN + (int)crank * 128 + r;
+      const bool n_ok = n < p.N;
+      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_lane + e * 128 + cc * 32, v);
+        tmem_ld_wait();
+        if (cc == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_on_leader(accempty, crank);
+        }
+        const int mb = tm * kQBT + e * 128 + cc * 32;
+        float sxl = 0.0f;
+        if (!OUT_I32 && mb + lane < p.M) sxl = __ldg(p.s_x + mb + lane);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int m = mb + i;
+          if constexpr (OUT_I32) {
+            if (m < p.M && n_ok) reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)v[i];
+          } else {
+            const float sx = __shfl_sync(0xffffffffu, sxl, i);
+            if (m < p.M && n_ok) {
+              const float y = __fmul_rn(__int2float_rn((int32_t)v[i]), __fmul_rn(sx, sc));
+              reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
+            }
+          }
+        }
+      }
+    }
+  epi_done:;
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // The even CTA's MMAs read the odd CTA's shared and tensor memory: neither
+  // CTA leaves before the pair is done.
+  __syncwarp();
+  tc_fence_before();
+  cluster_arrive();
+  cluster_wait();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
+}
+
+}  // namespace lq

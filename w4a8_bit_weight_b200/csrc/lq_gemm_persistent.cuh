@@ -8,15 +8,16 @@
 //     (token tiles fastest, so the CTAs in flight share weight tiles in L2);
 //   * two TMEM accumulators (2 x 128 columns) alternate between tiles, so the
 //     epilogue of tile j overlaps the mainloop of tile j+1;
-//   * eight expansion warps, two per TMEM lane quarter, each expanding one of
-//     the two 64-wide groups of a stage: the IMAD+XOR expansion of 128 x 128
-//     weights per stage has to keep pace with 256 cycles of tensor work.
+//   * kPExpGroups groups of four expansion warps; group g expands the stages
+//     of K-blocks g, g + kPExpGroups, ...  Expanding one stage (load, IMAD +
+//     XOR, tcgen05.st, wait for the store) takes longer than the 256 cycles
+//     of tensor work per stage, so several stages are expanded at once.
 //
-// Warp roles (448 threads):
+// Warp roles (64 + 128 * kPExpGroups + 128 threads):
 //   warp 0        TMA producer (one elected lane issues)
 //   warp 1        TMEM allocation, tcgen05.mma issue (one elected lane)
-//   warps 2-9     LiquidQuant expansion into the TMEM A slot of the stage
-//   warps 10-13   epilogue: TMEM accumulators -> scales -> bf16 stores
+//   warps 2..     LiquidQuant expansion into the TMEM A slot of the stage
+//   last 4 warps  epilogue: TMEM accumulators -> scales -> bf16 stores
 #pragma once
 
 #include <cuda_bf16.h>
@@ -28,7 +29,10 @@ namespace lq {
 
 constexpr int kPBT = 128;                 // tokens per tile
 constexpr int kPStages = 8;
-constexpr int kPThreads = 448;
+constexpr int kPExpGroups = 4;
+constexpr int kPEpiWarp0 = 2 + 4 * kPExpGroups;
+constexpr int kPThreads = 32 * (kPEpiWarp0 + 4);
+static_assert(kPStages % kPExpGroups == 0, "stages per expansion group");
 constexpr int kPXBytes = kPBT * kBlockK;  // 16 KB
 constexpr int kPWBytes = kBlockN * kBlockK / 2;
 constexpr int kPSABytes = 2 * kBlockN;
@@ -64,7 +68,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], 8);
+      mbar_init(&afull[s], 4);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -198,43 +202,43 @@ __global__ void __launch_bounds__(kPThreads, 1)
       while (!mbar_try_wait(a, 0) && globaltimer() - t0w < 100000000ull) {
       }
     }
-  } else if (warp < 10) {
+  } else if (warp < kPEpiWarp0) {
     // ------------------------------------------------------ expansion warps
     const int sub = warp & 3;
-    const int half = (warp - 2) >> 2;    // group 0 or 1 of the stage (64 k each)
+    const int grp = (warp - 2) >> 2;     // this group expands K-blocks grp, grp + G, ...
     const int r = sub * 32 + lane;       // weight row = TMEM lane
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     const int sw = (r >> 1) & 3;
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int tile = first_tile; tile < tiles; tile += stride) {
-      for (int kb = 0; kb < KB; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) goto exp_done;
-        tc_fence_after();
-        const uint8_t* sb = smem + stage * kPStageBytes;
-        const uint8_t* ss = sb + kPXBytes + kPWBytes;
-        const uint32_t s = ss[half * kBlockN + r];
-        const uint32_t a4 = (uint32_t)ss[kPSABytes + half * kBlockN + r] * 0x01010101u;
-        const uint32_t wrow = smem_u32(sb + kPXBytes) + r * (kBlockK / 2);
-        uint32_t v[16];
+    int ntiles = 0;
+    for (int tile = first_tile; tile < tiles; tile += stride) ++ntiles;
+    const int total = ntiles * KB;
+    for (int it = grp; it < total; it += kPExpGroups) {
+      const int stage = it % S;
+      const uint32_t phase = (uint32_t)(it / S) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) goto exp_done;
+      tc_fence_after();
+      const uint8_t* sb = smem + stage * kPStageBytes;
+      const uint8_t* ss = sb + kPXBytes + kPWBytes;
+      const uint32_t s0 = ss[r], s1 = ss[kBlockN + r];
+      const uint32_t a0 = (uint32_t)ss[kPSABytes + r] * 0x01010101u;
+      const uint32_t a1 = (uint32_t)ss[kPSABytes + kBlockN + r] * 0x01010101u;
+      const uint32_t wrow = smem_u32(sb + kPXBytes) + r * (kBlockK / 2);
+      uint32_t v[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint4 q = lds128(wrow + (((half * 2 + c) ^ sw) << 4));
-          lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
-          lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
-          lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
-          lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
-        }
-        tmem_st_32x32b_x16(t_lane + kPAccCols + stage * 32 + half * 16, v);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[stage]);
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
+      for (int c = 0; c < 4; ++c) {
+        const uint4 q = lds128(wrow + ((c ^ sw) << 4));
+        const uint32_t s = c < 2 ? s0 : s1;
+        const uint32_t a4 = c < 2 ? a0 : a1;
+        lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
+        lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
+        lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
+        lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
       }
+      tmem_st_32x32b_x32(t_lane + kPAccCols + stage * 32, v);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[stage]);
     }
   exp_done:;
   } else {
