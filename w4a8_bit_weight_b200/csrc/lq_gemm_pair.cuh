@@ -332,31 +332,66 @@ __global__ void __launch_bounds__(kQThreads, 1)
       const int n = tn * kQBN + (int)crank * 128 + r;
       const bool n_ok = n < p.N;
       const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
+      const int mb = tm * kQBT + e * 128;
+      if constexpr (OUT_I32) {
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(t_lane + e * 128 + cc * 32, v);
-        tmem_ld_wait();
-        if (cc == 3) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) arrive_on_leader(accempty, crank);
-        }
-        const int mb = tm * kQBT + e * 128 + cc * 32;
-        float sxl = 0.0f;
-        if (!OUT_I32 && mb + lane < p.M) sxl = __ldg(p.s_x + mb + lane);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int m = mb + i;
-          if constexpr (OUT_I32) {
-            if (m < p.M && n_ok) reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)v[i];
-          } else {
-            const float sx = __shfl_sync(0xffffffffu, sxl, i);
-            if (m < p.M && n_ok) {
-              const float y = __fmul_rn(__int2float_rn((int32_t)v[i]), __fmul_rn(sx, sc));
-              reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
-            }
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_lane + e * 128 + cc * 32, v);
+          tmem_ld_wait();
+          if (cc == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_on_leader(accempty, crank);
           }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int m = mb + cc * 32 + i;
+            if (m < p.M && n_ok) reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)v[i];
+          }
+        }
+      } else {
+        // All four chunks to packed bf16 in registers first, so the accumulator
+        // goes back to the MMA warp before any global store is issued.
+        uint32_t pk[64];  // pk[q] = bf16 pair for tokens (2q, 2q+1) of this warp's 128
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_lane + e * 128 + cc * 16, v);
+          const int m = mb + (cc >> 1) * 32 + lane;
+          const float sxl = (m < p.M) ? __ldg(p.s_x + m) : 0.0f;
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const int src = (cc & 1) * 16 + i;
+            const float s0 = __fmul_rn(__shfl_sync(0xffffffffu, sxl, src), sc);
+            const float s1 = __fmul_rn(__shfl_sync(0xffffffffu, sxl, src + 1), sc);
+            const float y0 = __fmul_rn(__int2float_rn((int32_t)v[i]), s0);
+            const float y1 = __fmul_rn(__int2float_rn((int32_t)v[i + 1]), s1);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+            pk[8 * cc + i / 2] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(accempty, crank);
+        // Stores: lanes 2j and 2j+1 swap halves so that each lane writes the two
+        // adjacent columns (n, n+1) of one token as one 4-byte word -- even
+        // lanes the even token of a pair, odd lanes the odd token.
+        const bool odd = lane & 1;
+        const int n0 = n & ~1;
+        const bool n0_ok = n0 < p.N;  // N is a multiple of 16, so n0 + 1 < N too
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          const uint32_t mine = pk[q];
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+          // even lane: (its token i at n, partner's token i at n+1); odd lane: token i+1
+          const uint32_t lo = odd ? (other >> 16) : (mine & 0xFFFFu);
+          const uint32_t hi = odd ? (mine >> 16) : (other & 0xFFFFu);
+          const int m = mb + 2 * q + (odd ? 1 : 0);
+          if (m < p.M && n0_ok)
+            *reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.N + n0) =
+                lo | (hi << 16);
         }
       }
     }
