@@ -56,25 +56,34 @@ template <int BT, int CS>
 struct GemmCfg {
   static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128 || BT == 256, "tokens per tile");
   static_assert(CS >= 0 && CS <= 8, "cluster size");
-  static constexpr int kStages = BT <= 64 ? 6 : (BT == 128 ? (CS >= 2 ? 6 : 8) : 5);
-  static constexpr int kXBytes = BT * kBlockK;             // int8 activation tile, 128-byte rows
-  static constexpr int kWBytes = kBlockN * kBlockK / 2;    // packed u4 weight tile, 64-byte rows
+  // shared-memory stages: a ring of activation tiles and a ring of weight tiles
+  static constexpr int kStages = BT <= 32 ? 8 : BT == 64 ? 6 : (BT == 128 ? (CS >= 2 ? 6 : 8) : 5);
+  static constexpr int kXBytes = BT * kBlockK;             // int8 activation tile, 128-byte rows (SW128)
+  static constexpr int kWBytes = kBlockN * kBlockK / 2;    // packed u4 weight tile, 64-byte rows (SW64)
   static constexpr int kSABytes = 2 * kBlockN;             // 2 groups x 128 rows of u8
-  static constexpr int kStageBytes = round_up_c(kXBytes + kWBytes + 2 * kSABytes, 1024);
-  static constexpr uint32_t kTxBytes = kXBytes + kWBytes + 2 * kSABytes;
-  static constexpr uint32_t kTxWeights = kWBytes + 2 * kSABytes;
+  static constexpr int kWStage = kWBytes + 2 * kSABytes;   // 8704 = 17 x 512: keeps the SW64 alignment
+  static constexpr uint32_t kTxX = kXBytes;
+  static constexpr uint32_t kTxW = kWStage;
   static constexpr int kAccCols = BT < 32 ? 32 : BT;      // int32 accumulator columns
-  static constexpr int kTmemCols = (kAccCols + kStages * 32 <= 256) ? 256 : 512;
+  // TMEM A slots (one expanded K-block of 128 each, 32 columns), independent of
+  // the number of shared-memory stages; small tiles keep to 256 columns so two
+  // CTAs can share an SM
+  static constexpr int kSlots = BT <= 64 ? (kStages < (256 - kAccCols) / 32 ? kStages : (256 - kAccCols) / 32)
+                                         : kStages;
+  static constexpr int kTmemCols = (kAccCols + kSlots * 32 <= 256) ? 256 : 512;
   static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * BT * kBlockN * 4 : 0;  // DSMEM partials
-  static constexpr int kBarBytes = 256;
-  static constexpr int kUsed = kStages * kStageBytes + kRedBytes + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kXRing = kStages * kXBytes;
+  static constexpr int kWRing = kStages * kWStage;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kUsed = kXRing + kWRing + kRedBytes + kBarBytes + 1024;  // + alignment slack
   // Shared memory also bounds how many CTAs share an SM: a 512-column CTA
   // takes at least 120 KB (one per SM), a 256-column CTA at least 80 KB (at
   // most two per SM), so co-resident CTAs never exceed the 512 TMEM columns.
   static constexpr int kSmemBytes = max_c(round_up_c(kUsed, 1024), kTmemCols == 512 ? 122880 : 81920);
-  static_assert(kAccCols + kStages * 32 <= kTmemCols, "TMEM budget");
+  static_assert(kAccCols + kSlots * 32 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(3 * kStages * 8 + 5 * 8 + 16 <= kBarBytes, "barrier area");
+  static_assert(kXBytes % 1024 == 0 && (kXRing + kWRing + kRedBytes) % 8 == 0, "alignment");
+  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 5 * 8 + 16 <= kBarBytes, "barrier area");
 };
 
 struct GemmArgs {
@@ -90,6 +99,14 @@ struct GemmArgs {
 
 __device__ __forceinline__ long long cta_of_unit(long long u, long long U, long long G) {
   return ((u + 1) * G + U - 1) / U - 1;
+}
+
+// One lane polls the barrier; the decision is broadcast to the warp (cheaper
+// than 32 lanes polling the same mbarrier).
+__device__ __forceinline__ bool lane0_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // Bounded barrier among the four epilogue warps (an mbarrier with count 4),
@@ -135,14 +152,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                      const GemmArgs p) {
   using C = GemmCfg<BT, CS>;
   constexpr int S = C::kStages;
+  constexpr int A = C::kSlots;
   constexpr int CH = BT < 32 ? BT : 32;  // accumulator columns per TMEM load
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int32_t* red = reinterpret_cast<int32_t*>(smem + S * C::kStageBytes);  // [CS-1][BT][128]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kRedBytes);
-  uint64_t* afull = full + S;
-  uint64_t* empty = afull + S;
-  uint64_t* accfull = empty + S;
+  uint8_t* xring = smem;                          // S x [BT][128] int8, SW128
+  uint8_t* wring = smem + C::kXRing;              // S x ([128][64] packed, SW64 | s [2][128] | a [2][128])
+  int32_t* red = reinterpret_cast<int32_t*>(smem + C::kXRing + C::kWRing);  // [CS-1][BT][128]
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::kXRing + C::kWRing + C::kRedBytes);
+  uint64_t* xfull = wfull + S;
+  uint64_t* empty = xfull + S;
+  uint64_t* afull = empty + S;    // [A]
+  uint64_t* aempty = afull + A;   // [A]
+  uint64_t* accfull = aempty + A;
   uint64_t* drain = accfull + 1;
   uint64_t* grp = drain + 1;
   uint64_t* redbar = grp + 1;
@@ -156,9 +178,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&afull[s], 4);
+      mbar_init(&wfull[s], 1);
+      mbar_init(&xfull[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < A; ++s) {
+      mbar_init(&afull[s], 4);
+      mbar_init(&aempty[s], 1);
     }
     mbar_init(accfull, 1);
     mbar_init(drain, 1);
@@ -205,98 +231,110 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = (lane == 0);
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Weight tiles depend on nothing the preceding kernel writes: the first
+    // S of them are requested before griddepcontrol.wait; activation tiles
+    // after it.  Weights and activations complete on separate barriers, so
+    // the expansion never waits for activations.
     uint64_t pol_stream = 0, pol_keep = 0;
     if (leader) {
       pol_stream = l2_policy_evict_first();  // weights: read once
       pol_keep = l2_policy_evict_last();     // activations: re-read per weight tile
     }
-    // weights of the first stages do not depend on the preceding kernel
-    const int t0 = (int)(u_begin / KB);
-    const int kbf = (int)(u_begin % KB);
-    const int P = (int)min((long long)S, min((long long)(KB - kbf), u_end - u_begin));
-    const int tn0 = t0 / p.tiles_m, tm0 = t0 % p.tiles_m;
+    const int total = (int)(u_end - u_begin);
+    const int P = min(S, total);
     if (leader) {
-      for (int i = 0; i < P; ++i) {
-        uint8_t* sb = smem + i * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[i], C::kTxBytes);
-        tma_load_2d(sb + C::kXBytes, &tm_w, &full[i], (kbf + i) * (kBlockK / 2), tn0 * kBlockN, pol_stream);
-        tma_load_2d(sb + C::kXBytes + C::kWBytes, &tm_s, &full[i], tn0 * kBlockN, (kbf + i) * 2, pol_stream);
-        tma_load_2d(sb + C::kXBytes + C::kWBytes + C::kSABytes, &tm_a, &full[i], tn0 * kBlockN, (kbf + i) * 2,
-                    pol_stream);
+      // first P K-blocks (they may span tiles in the stream-K schedule)
+      long long u = u_begin;
+      for (int i = 0; i < P; ++i, ++u) {
+        const int t = (int)(u / KB), kb = (int)(u % KB);
+        const int tile_n = t / p.tiles_m;
+        uint8_t* wb = wring + i * C::kWStage;
+        mbar_arrive_expect_tx(&wfull[i], C::kTxW);
+        tma_load_2d(wb, &tm_w, &wfull[i], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
+        tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], tile_n * kBlockN, kb * 2, pol_stream);
+        tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], tile_n * kBlockN, kb * 2, pol_stream);
       }
     }
     griddep_wait();
-    if (leader)
-      for (int i = 0; i < P; ++i)
-        tma_load_2d(smem + i * C::kStageBytes, &tm_x, &full[i], (kbf + i) * kBlockK, tm0 * BT, pol_keep);
+    if (leader) {
+      long long u = u_begin;
+      for (int i = 0; i < P; ++i, ++u) {
+        const int t = (int)(u / KB), kb = (int)(u % KB);
+        const int tile_m = t % p.tiles_m;
+        mbar_arrive_expect_tx(&xfull[i], C::kTxX);
+        tma_load_2d(xring + i * C::kXBytes, &tm_x, &xfull[i], kb * kBlockK, tile_m * BT, pol_keep);
+      }
+    }
     __syncwarp();
-    int stage = 0;
-    uint32_t phase = 0;
     uint32_t issued = P >= 32 ? 0xffffffffu : ((1u << P) - 1u), issued_par = 0;
-    int it = 0;
-    for (long long u = u_begin; u < u_end;) {
-      const int t = (int)(u / KB);
-      const int kb0 = (int)(u % KB);
-      const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
-      const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
-      for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        if (it >= P) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1u, abort_flag))) goto producer_done;
-          if (leader) {
-            uint8_t* sb = smem + stage * C::kStageBytes;
-            mbar_arrive_expect_tx(&full[stage], C::kTxBytes);
-            tma_load_2d(sb, &tm_x, &full[stage], kb * kBlockK, tile_m * BT, pol_keep);
-            tma_load_2d(sb + C::kXBytes, &tm_w, &full[stage], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
-            tma_load_2d(sb + C::kXBytes + C::kWBytes, &tm_s, &full[stage], tile_n * kBlockN, kb * 2, pol_stream);
-            tma_load_2d(sb + C::kXBytes + C::kWBytes + C::kSABytes, &tm_a, &full[stage], tile_n * kBlockN, kb * 2,
-                        pol_stream);
-          }
-          issued |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+    {
+      int stage = P % S;
+      uint32_t phase = (uint32_t)(P / S) & 1u;
+      long long u = u_begin + P;
+      for (int it = P; it < total; ++it, ++u) {
+        if (!lane0_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
+        if (leader) {
+          const int t = (int)(u / KB), kb = (int)(u % KB);
+          const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
+          uint8_t* wb = wring + stage * C::kWStage;
+          mbar_arrive_expect_tx(&wfull[stage], C::kTxW);
+          tma_load_2d(wb, &tm_w, &wfull[stage], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
+          tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[stage], tile_n * kBlockN, kb * 2, pol_stream);
+          tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[stage], tile_n * kBlockN, kb * 2, pol_stream);
+          mbar_arrive_expect_tx(&xfull[stage], C::kTxX);
+          tma_load_2d(xring + stage * C::kXBytes, &tm_x, &xfull[stage], kb * kBlockK, tile_m * BT, pol_keep);
         }
+        issued |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      u += kb1 - kb0;
     }
   producer_done:
     if (leader && *abort_flag) {
       // never leave a bulk copy in flight into shared memory that is about to be released
       for (int s = 0; s < S; ++s)
         if (issued & (1u << s)) {
-          const uint32_t a = smem_u32(&full[s]);
           const unsigned long long t0w = globaltimer();
-          while (!mbar_try_wait(a, (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
+          while (!mbar_try_wait(smem_u32(&wfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
+          }
+          while (!mbar_try_wait(smem_u32(&xfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
           }
         }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = idesc_i8(BT);
-    int stage = 0;
-    uint32_t phase = 0;
     bool any = false;
+    int stage = 0, slot = 0;
+    uint32_t sphase = 0, aphase = 0;
     for (long long u = u_begin; u < u_end;) {
       const int kb0 = (int)(u % KB);
       const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&afull[stage], phase, abort_flag))) goto mma_done;
-        tc_fence_after();
+        bool ok = true;
+        if (leader) ok = mbar_wait(&afull[slot], aphase, abort_flag) && mbar_wait(&xfull[stage], sphase, abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) goto mma_done;
         if (leader) {
-          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(smem + stage * C::kStageBytes));
-          const uint32_t a_col = tmem_base + C::kAccCols + stage * 32;
+          tc_fence_after();
+          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
+          const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
 #pragma unroll
           for (int j = 0; j < kBlockK / 32; ++j)
             mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb > kb0 || j > 0) ? 1u : 0u);
           tc_commit(&empty[stage]);
+          tc_commit(&aempty[slot]);
         }
-        __syncwarp();
         any = true;
         if (++stage == S) {
           stage = 0;
-          phase ^= 1u;
+          sphase ^= 1u;
+        }
+        if (++slot == A) {
+          slot = 0;
+          aphase ^= 1u;
         }
       }
       if (leader) tc_commit(accfull);
@@ -320,10 +358,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = sub * 32 + lane;      // weight row of the tile = TMEM lane
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     const int sw = (r >> 1) & 3;        // 64-byte swizzle of this row's 16-byte chunks
-    int stage = 0;
-    uint32_t phase = 0, acc_phase = 0, grp_phase = 0;
+    uint32_t acc_phase = 0, grp_phase = 0;
     bool waited_dep = false;
     bool red_done = (CS < 2 || crank != 0);
+    int stage = 0, slot = 0;
+    uint32_t sphase = 0, aphase = 0;
     for (long long u = u_begin; u < u_end;) {
       const int t = (int)(u / KB);
       const int kb0 = (int)(u % KB);
@@ -331,14 +370,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
       for (int kb = kb0; kb < kb1; ++kb) {
         // warp-uniform decision: every lane waits, all continue only if all saw the phase
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag))) goto epi_done;
+        if (!__all_sync(0xffffffffu, mbar_wait(&wfull[stage], sphase, abort_flag) &&
+                                         mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag)))
+          goto epi_done;
         tc_fence_after();
-        const uint8_t* sb = smem + stage * C::kStageBytes;
-        const uint8_t* ss = sb + C::kXBytes + C::kWBytes;
+        const uint8_t* wb = wring + stage * C::kWStage;
+        const uint8_t* ss = wb + C::kWBytes;
         const uint8_t* sa = ss + C::kSABytes;
         const uint32_t s0 = ss[r], s1 = ss[kBlockN + r];
         const uint32_t a0 = (uint32_t)sa[r] * 0x01010101u, a1 = (uint32_t)sa[kBlockN + r] * 0x01010101u;
-        const uint32_t wrow = smem_u32(sb + C::kXBytes) + r * (kBlockK / 2);
+        const uint32_t wrow = smem_u32(wb) + r * (kBlockK / 2);
         uint32_t v[32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -350,14 +391,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
           lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
         }
-        tmem_st_32x32b_x32(t_lane + C::kAccCols + stage * 32, v);
+        tmem_st_32x32b_x32(t_lane + C::kAccCols + slot * 32, v);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[stage]);
+        if (lane == 0) mbar_arrive(&afull[slot]);
         if (++stage == S) {
           stage = 0;
-          phase ^= 1u;
+          sphase ^= 1u;
+        }
+        if (++slot == A) {
+          slot = 0;
+          aphase ^= 1u;
         }
       }
 
