@@ -199,6 +199,33 @@ LQ_API lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, c
                                 int K, int group, int8_t* w_i8, void* stream);
 
 /*
+ * lq_w4a8_gemm_noalloc -- lq_w4a8_gemm for callers that must not allocate
+ * device memory where they launch the GEMM (a serving framework's enqueue
+ * hook that owns all device memory, a latency-critical loop that cannot block
+ * on the allocator or fail on out-of-memory mid-request).  The paper has no
+ * counterpart; this is an interface convenience of this library.
+ *   Same operands, layouts and result as lq_w4a8_gemm, computed with the
+ *   stream-K schedule (one CTA per SM).  Its partial sums live in a 4 MiB
+ *   scratch array inside the library image (held on every GPU that loads the
+ *   library until the process exits) instead of a workspace; nothing is
+ *   allocated and no workspace is passed.
+ *   The scratch needed is ceil(M/bt) * ceil(N/128) * bt * 512 bytes plus a
+ *   small tile counter area, bt being the automatic token-tile width (16, 32,
+ *   64 or 128 tokens for M <= 16, 32, 64, larger); shapes that need more than
+ *   the array return LQ_ERR_WORKSPACE without launching anything.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  Every call clears the part of the array it
+ *   uses (an asynchronous memset on `stream`) before the GEMM.
+ *   All calls on a device share the one array: calls that can overlap on the
+ *   GPU race and corrupt each other's results, so order them (e.g. issue
+ *   them on one stream).
+ */
+LQ_API lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                                      const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c,
+                                      void* out_bf16, int M, int N, int K, int group, void* stream);
+
+/*
  * lq_get_device_error -- synchronizes `stream`, then reads and clears the
  * library's device error word.  Returns LQ_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last call (its output is then undefined),

@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_gemm_i32": ([P, P, P, P, P, I, I, I, I, P, Z, P], I),
             "lq_dequant_weights_i8": ([P, P, P, I, I, I, P, P], I),
             "lq_get_device_error": ([P], I),
+            "lq_w4a8_gemm_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -231,6 +232,29 @@ def lq_w4a8_gemm_i32(x_q, qw, s_u8, a_u8, out=None, group: int = GROUP, block_t:
     """The int32 accumulators x_q @ dequant(qw)^T -> [M, N] int32."""
     return _gemm(x_q, None, qw, s_u8, a_u8, None, out, group, block_t, split_k, grid, True, workspace_buf,
                  schedule)
+
+
+def lq_w4a8_gemm_noalloc(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP):
+    """lq_w4a8_gemm without a workspace, for callers that may not allocate device memory
+    where they launch the GEMM; its scratch is a fixed 4 MiB array inside the library.
+    Calls on one device share that array and must not overlap on the GPU."""
+    lib = load_library()
+    _need(x_q, torch.int8, "x_q")
+    M, K = x_q.shape
+    N = qw.shape[0]
+    _need(qw, torch.uint8, "qw", (N, K // 2))
+    _need(s_u8, torch.uint8, "s_u8", (K // group, N))
+    _need(a_u8, torch.uint8, "a_u8", (K // group, N))
+    _need(s_x, torch.float32, "s_x", (M,))
+    _need(s_c, torch.float32, "s_c", (N,))
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x_q.device)
+    _need(out, torch.bfloat16, "out", (M, N))
+    with torch.cuda.device(x_q.device):
+        _check("lq_w4a8_gemm_noalloc", lib.lq_w4a8_gemm_noalloc(
+            _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out),
+            M, N, K, group, _stream(x_q.device)))
+    return out
 
 
 def lq_dequant_weights_i8(qw, s_u8, a_u8, group: int = GROUP, out=None):

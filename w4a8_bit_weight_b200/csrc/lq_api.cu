@@ -479,3 +479,76 @@ lq_status lq_get_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free GEMM.
+//
+// Some callers may not allocate device memory on the path that launches the
+// GEMM: a serving framework's per-request enqueue hook (the framework owns all
+// device memory and does not expect a library to call cudaMalloc there), or a
+// latency-critical loop that must not block on the driver's allocator or fail
+// on an out-of-memory error mid-request.  lq_w4a8_gemm_noalloc serves them: it
+// runs the stream-K schedule with its int32 partial sums and tile tickets in
+// the fixed array below instead of a caller-provided workspace.
+//
+// The array is part of the library image: every GPU on which the library is
+// loaded holds these kNoAllocScratchBytes until the process exits.  All calls
+// on a device share it, so two calls that overlap on the GPU (different
+// streams, or one stream racing another) corrupt each other's sums; callers
+// must order them, e.g. on a single stream.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, resolved once per device.  In host code
+// the array's name only stands for the symbol; kernels must be given this
+// address.
+void* g_noalloc_addr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+lq_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LQ_ERR_CUDA;
+  if (!g_noalloc_addr[dev]) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LQ_ERR_CUDA;
+      g_noalloc_addr[dev] = p;
+    }
+  }
+  *out = g_noalloc_addr[dev];
+  return LQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                               const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K,
+                               int group, void* stream) {
+  lq_status st = check_gemm_shape(M, N, K, group);
+  if (st != LQ_OK) return st;
+  if (M == 0) return LQ_OK;
+  if (!x_q || !qw || !s_u8 || !a_u8 || !out_bf16 || !s_x || !s_c) return LQ_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  const Schedule s = make_schedule(M, N, K, 0, kSchedStreamK, 0, 0, dev->sms);
+  if (s.ws_bytes > kNoAllocScratchBytes) return LQ_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != LQ_OK) return st;
+  // the partial sums and tickets start from zero on every call, whatever an
+  // earlier (possibly failed) call left behind
+  if (s.ws_bytes != 0 &&
+      cudaMemsetAsync(scratch, 0, s.ws_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, scratch, kNoAllocScratchBytes, 0,
+                   kSchedStreamK, 0, 0, false, stream);
+}
+
+}  // extern "C"
