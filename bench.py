@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--soak-s", type=float, default=1.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill measurement of the default run")
     return ap.parse_args()
 
 
@@ -110,6 +111,15 @@ def ncu_traffic(workload):
     if not e or e.get("kernel_source") != kernel_source_hash():
         return None
     return e.get("dram_bytes_per_gemm_launch")
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    """Max of `value` over all ranks (the slowest rank sets the job's time)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ---------------------------------------------------------------------------
@@ -305,12 +315,7 @@ def run_ours(args, rank, world, local_rank):
         graph.replay()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return reduce_max(e0.elapsed_time(e1), world, dev)
 
     with torch.cuda.stream(stream):
         ms_total = timed(g_timed)
@@ -384,8 +389,87 @@ def run_ours(args, rank, world, local_rank):
                       "how": "pinned host X -> device copy, quantize_act + gemm, device -> pinned host out, "
                              "per M, same CUDA graph method"}
     res["int8_peak_tops"] = int8_peak
+    if args.workload == "decode" and not args.no_secondary:
+        pre = secondary_workload("prefill", dev)
+        g = pre["4096"]
+        pre["roofline"] = {"bound": "tensor", "kernel": "w4a8_gemm_pair_kernel", "achieved": g["gemm_tops"],
+                           "peak": int8_peak, "unit": "TOPS", "frac": g["gemm_tops"] / int8_peak,
+                           "peak_source": f"{pk_src}: {INT8_OVER_BF16:g} x bf16 burst",
+                           "frac_of_nominal_4500": g["gemm_tops"] / 4500.0,
+                           "traffic": ncu_traffic("prefill")}
+        res["prefill"] = pre
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w)
+    return res
+
+
+def secondary_workload(name, dev, steps=20):
+    """A short measurement of another workload in the same run (the metric also names
+    prefill M=4096): K steps of act-quant + GEMM in one CUDA graph, then the GEMM's own
+    duration from events around each GEMM node of a second replay."""
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+    w = synth.WORKLOADS[name]
+    X, W = synth.make_workload(w)
+    qw, s_u8, a_u8, s_c = lq.lq_quantize_weights(W.to(dev))
+    wset_bytes = qw.numel() + s_u8.numel() + a_u8.numel() + 4 * s_c.numel()
+    n_sets = min(64, max(4, int(np.ceil(3 * L2_BYTES / wset_bytes))))
+    sets = [(qw, s_u8, a_u8, s_c)] + [(qw.clone(), s_u8.clone(), a_u8.clone(), s_c.clone())
+                                      for _ in range(n_sets - 1)]
+    Xd = X.to(dev)
+    res = {"workload": w.note}
+    stream = torch.cuda.Stream(dev)
+    for M in w.Ms:
+        xq = torch.empty(M, w.K, dtype=torch.int8, device=dev)
+        sx = torch.empty(M, dtype=torch.float32, device=dev)
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
+        cnt = [0]
+        evs = []
+
+        def one(events=None):
+            lq.lq_quantize_act(Xd[:M], out=(xq, sx))
+            wq = sets[cnt[0] % n_sets]
+            cnt[0] += 1
+            if events is None:
+                lq.lq_w4a8_gemm(xq, sx, *wq, out=out)
+            else:
+                e0 = torch.cuda.Event(enable_timing=True, external=True)
+                e1 = torch.cuda.Event(enable_timing=True, external=True)
+                e0.record()
+                lq.lq_w4a8_gemm(xq, sx, *wq, out=out)
+                e1.record()
+                events.append((e0, e1))
+
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                one()
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(steps):
+                    one()
+            gi = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gi, stream=stream):
+                for _ in range(steps):
+                    one(evs)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = a.elapsed_time(b) / steps
+            gi.replay()
+            torch.cuda.synchronize(dev)
+        gemm_ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+        ops = 2.0 * M * w.N * w.K
+        res[str(M)] = {"ms_per_step": ms, "tops_step": ops / (ms * 1e-3) / 1e12,
+                       "gemm_us": 1e3 * gemm_ms, "gemm_tops": ops / (gemm_ms * 1e-3) / 1e12,
+                       "gemm_gbs": gemm_bytes(M, w.N, w.K) / (gemm_ms * 1e-3) / 1e9}
+    st = lq.lq_get_device_error(dev)
+    if st != 0:
+        raise RuntimeError(f"device error in the {name} measurement: {st}")
     return res
 
 
