@@ -13,22 +13,29 @@
 //     all 256 tokens;
 //   * one thread of the even CTA issues every MMA for both SMs: 128 cycles of
 //     tensor work per SM per instruction, enough to hide the issue cost.
-// Stages carry 256 K (four groups of 64).  The accumulator is single: the
-// epilogue warps of both CTAs hand it back as soon as their last TMEM load
-// has landed, so only the loads (not the stores) sit between two tiles.
+// Stages carry 256 K (four groups of 64) and come in two rings: weight
+// stages (packed codes, scales, offsets) are released as soon as the
+// expansion warps have read them, activation stages when the MMAs that read
+// them complete -- so refilling weights never waits for the tensor core and
+// expansion stays off the activation refill path.  The accumulator is single:
+// the epilogue warps of both CTAs hand it back as soon as it sits in their
+// registers as packed bf16, before any global store.
 //
 // Hand-offs between the two CTAs:
-//   expansion done  -> arrive on the even CTA's afull[stage] (remote for odd)
-//   stage consumed  -> tcgen05.commit multicast to empty[stage] of both CTAs
-//   tile finished   -> tcgen05.commit multicast to accfull of both CTAs
-//   accum. loaded   -> arrive on the even CTA's accempty (remote for odd)
+//   activations landed (odd) -> forwarded to the even CTA's xpeer[stage]
+//   expansion done            -> arrive on the even CTA's afull[slot] (remote for odd)
+//   stage consumed            -> tcgen05.commit multicast to xempty/aempty of both CTAs
+//   tile finished             -> tcgen05.commit multicast to accfull of both CTAs
+//   accumulator loaded        -> arrive on the even CTA's accempty (remote for odd)
 // No TMA load uses cluster multicast: each CTA loads its own data.
 //
-// Warp roles (576 threads):
-//   warp 0        TMA producer
-//   warp 1        TMEM allocation (both CTAs); MMA issue (even CTA)
-//   warps 2-9     expansion: two groups of four warps, alternate stages
+// Warp roles (608 threads):
+//   warp 0        TMA producer of weight stages
+//   warp 1        TMEM allocation (both CTAs); MMA issue (even CTA);
+//                 activation-ready forwarding (odd CTA)
+//   warps 2-9     expansion: two groups of four warps, alternate K-blocks
 //   warps 10-17   epilogue: two warps per TMEM lane quarter, 128 tokens each
+//   warp 18       TMA producer of activation stages
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,23 +48,30 @@ namespace lq {
 constexpr int kQBT = 256;                     // tokens per tile (MMA N)
 constexpr int kQBN = 256;                     // weight rows per tile (MMA M, 128 per CTA)
 constexpr int kQBK = 256;                     // K per stage
-constexpr int kQStages = 4;
+constexpr int kQXStages = 4;                  // activation ring
+constexpr int kQWStages = 5;                  // weight ring
+constexpr int kQSlots = 4;                    // TMEM A slots
 constexpr int kQExpGroups = 2;
 constexpr int kQEpiWarp0 = 2 + 4 * kQExpGroups;
-constexpr int kQThreads = 32 * (kQEpiWarp0 + 8);
+constexpr int kQXProdWarp = kQEpiWarp0 + 8;
+constexpr int kQThreads = 32 * (kQXProdWarp + 1);
 constexpr int kQXSub = 128 * 128;             // one 128-token x 128-K SW128 sub-tile
 constexpr int kQXBytes = 2 * kQXSub;          // 32 KB: this CTA's 128 tokens x 256 K
-constexpr int kQWBytes = 128 * kQBK / 2;      // 16 KB: 128 rows x 256 codes, 128-byte rows
+constexpr int kQWBytes = 128 * kQBK / 2;      // 16 KB: 128 rows x 256 codes, 128-byte rows (SW128)
 constexpr int kQSABytes = (kQBK / 64) * 128;  // 4 groups x 128 rows
-constexpr int kQStageBytes = round_up_c(kQXBytes + kQWBytes + 2 * kQSABytes, 1024);
-constexpr uint32_t kQTx = kQXBytes + kQWBytes + 2 * kQSABytes;
+constexpr int kQWStage = kQWBytes + 2 * kQSABytes;  // 17 KB, keeps the 1024-byte alignment
+constexpr uint32_t kQTxX = kQXBytes;
+constexpr uint32_t kQTxW = kQWStage;
 constexpr int kQAccCols = kQBT;               // one accumulator
 constexpr int kQSlotCols = kQBK / 4;          // 64 TMEM columns per expanded stage
-constexpr int kQBarBytes = 256;
-constexpr int kQSmemBytes = kQStages * kQStageBytes + kQBarBytes + 1024;
-static_assert(kQAccCols + kQStages * kQSlotCols <= 512, "TMEM budget");
+constexpr int kQXRing = kQXStages * kQXBytes;
+constexpr int kQWRing = kQWStages * kQWStage;
+constexpr int kQBarBytes = 512;
+constexpr int kQSmemBytes = kQXRing + kQWRing + kQBarBytes + 1024;
+static_assert(kQWStage % 1024 == 0, "weight stage alignment");
+static_assert(kQAccCols + kQSlots * kQSlotCols <= 512, "TMEM budget");
 static_assert(kQSmemBytes <= 232448, "shared memory budget");
-static_assert(kQStages % kQExpGroups == 0, "stages per expansion group");
+static_assert(kQSlots % kQExpGroups == 0, "slots per expansion group");
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -113,13 +127,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
     w4a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                           const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
                           const GemmArgs p) {
-  constexpr int S = kQStages;
+  constexpr int SX = kQXStages, SW = kQWStages, A = kQSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kQStageBytes);
-  uint64_t* afull = full + S;
-  uint64_t* empty = afull + S;
-  uint64_t* accfull = empty + S;
+  uint8_t* xring = smem;                 // SX x [2][128 tokens][128 B], SW128
+  uint8_t* wring = smem + kQXRing;       // SW x ([128 rows][128 B] SW128 | s [4][128] | a [4][128])
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + kQXRing + kQWRing);
+  uint64_t* xpeer = xfull + SX;          // even CTA: the odd CTA's activations have landed
+  uint64_t* xempty = xpeer + SX;
+  uint64_t* wfull = xempty + SX;
+  uint64_t* wempty = wfull + SW;
+  uint64_t* afull = wempty + SW;         // [A]
+  uint64_t* aempty = afull + A;          // [A]
+  uint64_t* accfull = aempty + A;
   uint64_t* accempty = accfull + 1;
   uint64_t* drain = accempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -132,10 +152,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const bool even = (crank == 0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xpeer[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 4);  // the four warps of the expansion group that read it
+    }
+    for (int s = 0; s < A; ++s) {
       mbar_init(&afull[s], 8);   // four expansion warps of each CTA
-      mbar_init(&empty[s], 1);
+      mbar_init(&aempty[s], 1);
     }
     mbar_init(accfull, 1);
     mbar_init(accempty, 16);     // eight epilogue warps of each CTA
@@ -164,103 +192,104 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int tiles = (int)(p.U);             // host passes the tile count in U
   const int cid = blockIdx.x >> 1;
   const int ncl = gridDim.x >> 1;
+  int ntiles = 0;
+  for (int tile = cid; tile < tiles; tile += ncl) ++ntiles;
+  const int total = ntiles * KS;            // K-blocks this CTA takes part in
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    uint64_t pol_stream = 0, pol_keep = 0;
-    if (leader) {
-      pol_stream = l2_policy_evict_first();
-      pol_keep = l2_policy_evict_last();
-    }
-    const int P = cid < tiles ? min(S, KS) : 0;
-    const int t0n = cid / tiles_m, t0m = cid % tiles_m;
-    if (leader)
-      for (int i = 0; i < P; ++i) {
-        uint8_t* sb = smem + i * kQStageBytes;
-        mbar_arrive_expect_tx(&full[i], kQTx);
-        tma_load_2d(sb + kQXBytes, &tm_w, &full[i], i * (kQBK / 2), t0n * kQBN + (int)crank * 128, pol_stream);
-        tma_load_2d(sb + kQXBytes + kQWBytes, &tm_s, &full[i], t0n * kQBN + (int)crank * 128, i * 4, pol_stream);
-        tma_load_2d(sb + kQXBytes + kQWBytes + kQSABytes, &tm_a, &full[i], t0n * kQBN + (int)crank * 128, i * 4,
-                    pol_stream);
-      }
-    griddep_wait();
-    if (leader)
-      for (int i = 0; i < P; ++i) {
-        uint8_t* sb = smem + i * kQStageBytes;
-        tma_load_2d(sb, &tm_x, &full[i], i * kQBK, t0m * kQBT + (int)crank * 128, pol_keep);
-        tma_load_2d(sb + kQXSub, &tm_x, &full[i], i * kQBK + 128, t0m * kQBT + (int)crank * 128, pol_keep);
-      }
-    __syncwarp();
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued = (1u << P) - 1u, issued_par = 0;
+    // ---------------------------------------------------- weight producer
+    // weights depend on nothing the preceding kernel writes: no dependency wait
+    uint64_t pol = 0;
+    if (leader) pol = l2_policy_evict_first();
+    uint32_t issued = 0, issued_par = 0;
     int it = 0;
     for (int tile = cid; tile < tiles; tile += ncl) {
-      const int tm = tile % tiles_m, tn = tile / tiles_m;
-      const int xrow = tm * kQBT + (int)crank * 128;
-      const int wrow = tn * kQBN + (int)crank * 128;
+      const int wrow = (tile / tiles_m) * kQBN + (int)crank * 128;
       for (int kb = 0; kb < KS; ++kb, ++it) {
-        if (it >= P) {
-          if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, false)) goto producer_done;
-          if (leader) {
-            uint8_t* sb = smem + stage * kQStageBytes;
-            mbar_arrive_expect_tx(&full[stage], kQTx);
-            tma_load_2d(sb, &tm_x, &full[stage], kb * kQBK, xrow, pol_keep);
-            tma_load_2d(sb + kQXSub, &tm_x, &full[stage], kb * kQBK + 128, xrow, pol_keep);
-            tma_load_2d(sb + kQXBytes, &tm_w, &full[stage], kb * (kQBK / 2), wrow, pol_stream);
-            tma_load_2d(sb + kQXBytes + kQWBytes, &tm_s, &full[stage], wrow, kb * 4, pol_stream);
-            tma_load_2d(sb + kQXBytes + kQWBytes + kQSABytes, &tm_a, &full[stage], wrow, kb * 4, pol_stream);
-          }
-          issued |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        const int w = it % SW;
+        const uint32_t use = (uint32_t)(it / SW);
+        if (it >= SW && !warp_wait(&wempty[w], (use & 1u) ^ 1u, abort_flag, false)) goto wprod_done;
+        if (leader) {
+          uint8_t* wb = wring + w * kQWStage;
+          mbar_arrive_expect_tx(&wfull[w], kQTxW);
+          tma_load_2d(wb, &tm_w, &wfull[w], kb * (kQBK / 2), wrow, pol);
+          tma_load_2d(wb + kQWBytes, &tm_s, &wfull[w], wrow, kb * 4, pol);
+          tma_load_2d(wb + kQWBytes + kQSABytes, &tm_a, &wfull[w], wrow, kb * 4, pol);
         }
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        issued |= 1u << w;
+        issued_par = (issued_par & ~(1u << w)) | ((use & 1u) << w);
       }
     }
-  producer_done:
-    if (leader && *abort_flag) {
-      for (int s = 0; s < S; ++s)
+  wprod_done:
+    if (leader && *abort_flag)
+      for (int s = 0; s < SW; ++s)
         if (issued & (1u << s)) {
-          const uint32_t a = smem_u32(&full[s]);
           const unsigned long long t0w = globaltimer();
-          while (!mbar_try_wait(a, (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
+          while (!mbar_try_wait(smem_u32(&wfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
           }
         }
+  } else if (warp == kQXProdWarp) {
+    // ------------------------------------------------ activation producer
+    uint64_t pol = 0;
+    if (leader) pol = l2_policy_evict_last();
+    griddep_wait();  // activations may be the output of the preceding kernel
+    uint32_t issued = 0, issued_par = 0;
+    int it = 0;
+    for (int tile = cid; tile < tiles; tile += ncl) {
+      const int xrow = (tile % tiles_m) * kQBT + (int)crank * 128;
+      for (int kb = 0; kb < KS; ++kb, ++it) {
+        const int x = it % SX;
+        const uint32_t use = (uint32_t)(it / SX);
+        if (it >= SX && !warp_wait(&xempty[x], (use & 1u) ^ 1u, abort_flag, false)) goto xprod_done;
+        if (leader) {
+          uint8_t* xb = xring + x * kQXBytes;
+          mbar_arrive_expect_tx(&xfull[x], kQTxX);
+          tma_load_2d(xb, &tm_x, &xfull[x], kb * kQBK, xrow, pol);
+          tma_load_2d(xb + kQXSub, &tm_x, &xfull[x], kb * kQBK + 128, xrow, pol);
+        }
+        issued |= 1u << x;
+        issued_par = (issued_par & ~(1u << x)) | ((use & 1u) << x);
+      }
     }
+  xprod_done:
+    if (leader && *abort_flag)
+      for (int s = 0; s < SX; ++s)
+        if (issued & (1u << s)) {
+          const unsigned long long t0w = globaltimer();
+          while (!mbar_try_wait(smem_u32(&xfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
+          }
+        }
   } else if (warp == 1) {
-    // ------------------------------------------------- MMA issuer (even CTA)
     if (even) {
+      // ------------------------------------------------- MMA issuer (even CTA)
       const uint32_t idesc = idesc_i8_pair();
-      int stage = 0;
-      uint32_t phase = 0;
       bool any = false;
-      int j = 0;
+      int it = 0, j = 0;
       for (int tile = cid; tile < tiles; tile += ncl, ++j) {
         // the single accumulator is free once both CTAs' epilogues have loaded it
         if (!warp_wait(accempty, ((uint32_t)j & 1u) ^ 1u, abort_flag, true)) goto mma_done;
         tc_fence_after();
-        for (int kb = 0; kb < KS; ++kb) {
-          if (!warp_wait(&afull[stage], phase, abort_flag, true)) goto mma_done;
-          tc_fence_after();
+        for (int kb = 0; kb < KS; ++kb, ++it) {
+          const int x = it % SX, slot = it % A;
+          const uint32_t xpar = (uint32_t)(it / SX) & 1u, apar = (uint32_t)(it / A) & 1u;
+          bool ok = true;
+          if (leader)
+            ok = mbar_wait_cluster(&afull[slot], apar, abort_flag) && mbar_wait(&xfull[x], xpar, abort_flag) &&
+                 mbar_wait_cluster(&xpeer[x], xpar, abort_flag);
+          if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) goto mma_done;
           if (leader) {
-            const uint32_t xs = smem_u32(smem + stage * kQStageBytes);
-            const uint32_t a_col = tmem_base + kQAccCols + stage * kQSlotCols;
+            tc_fence_after();
+            const uint32_t xs = smem_u32(xring + x * kQXBytes);
+            const uint32_t a_col = tmem_base + kQAccCols + slot * kQSlotCols;
 #pragma unroll
             for (int jj = 0; jj < kQBK / 32; ++jj) {
               const uint64_t bdesc = smem_desc_k_sw128(xs + (jj >> 2) * kQXSub) + (uint64_t)(2 * (jj & 3));
               mma_i8_ts_pair(tmem_base, a_col + jj * 8, bdesc, idesc, (kb > 0 || jj > 0) ? 1u : 0u);
             }
-            tc_commit_pair_mc(&empty[stage], 0x3);
+            tc_commit_pair_mc(&xempty[x], 0x3);
+            tc_commit_pair_mc(&aempty[slot], 0x3);
           }
-          __syncwarp();
           any = true;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
         if (leader) tc_commit_pair_mc(accfull, 0x3);
         __syncwarp();
@@ -274,6 +303,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         while (!mbar_try_wait(a, 0) && globaltimer() - t0w < 100000000ull) {
         }
       }
+    } else {
+      // -------------------------- odd CTA: forward "activations landed" to the even CTA
+      const uint32_t peer_xpeer = mapa_shared(smem_u32(xpeer), 0);
+      for (int it = 0; it < total; ++it) {
+        const int x = it % SX;
+        if (!warp_wait(&xfull[x], (uint32_t)(it / SX) & 1u, abort_flag, false)) break;
+        if (leader) mbar_arrive_remote(peer_xpeer + (uint32_t)(x * 8));
+      }
     }
   } else if (warp < kQEpiWarp0) {
     // ------------------------------------------------------ expansion warps
@@ -282,23 +319,22 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const int r = sub * 32 + lane;
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     const int sw = r & 7;                // 128-byte swizzle of this row's 16-byte chunks
-    int ntiles = 0;
-    for (int tile = cid; tile < tiles; tile += ncl) ++ntiles;
-    const int total = ntiles * KS;
     for (int it = grp; it < total; it += kQExpGroups) {
-      const int stage = it % S;
-      const uint32_t phase = (uint32_t)(it / S) & 1u;
-      if (!warp_wait(&full[stage], phase, abort_flag, false)) goto exp_done;
+      const int w = it % SW, slot = it % A;
+      if (!__all_sync(0xffffffffu, mbar_wait(&wfull[w], (uint32_t)(it / SW) & 1u, abort_flag) &&
+                                       mbar_wait(&aempty[slot], ((uint32_t)(it / A) & 1u) ^ 1u, abort_flag)))
+        goto exp_done;
       tc_fence_after();
-      const uint8_t* sb = smem + stage * kQStageBytes;
-      const uint8_t* ss = sb + kQXBytes + kQWBytes;
-      const uint32_t wrow = smem_u32(sb + kQXBytes) + r * (kQBK / 2);
+      const uint8_t* wb = wring + w * kQWStage;
+      const uint8_t* ss = wb + kQWBytes;
+      const uint32_t wrow = smem_u32(wb) + r * (kQBK / 2);
+      uint32_t v0[32], v1[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {        // 128 K per half: groups 2h, 2h+1
         const uint32_t s0 = ss[(2 * h) * 128 + r], s1 = ss[(2 * h + 1) * 128 + r];
         const uint32_t a0 = (uint32_t)ss[kQSABytes + (2 * h) * 128 + r] * 0x01010101u;
         const uint32_t a1 = (uint32_t)ss[kQSABytes + (2 * h + 1) * 128 + r] * 0x01010101u;
-        uint32_t v[32];
+        uint32_t* v = h ? v1 : v0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint4 q = lds128(wrow + (((4 * h + c) ^ sw) << 4));
@@ -309,12 +345,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
           lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
           lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
         }
-        tmem_st_32x32b_x32(t_lane + kQAccCols + stage * kQSlotCols + h * 32, v);
       }
+      // the weight stage has been read: the producer may refill it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wempty[w]);
+      tmem_st_32x32b_x32(t_lane + kQAccCols + slot * kQSlotCols, v0);
+      tmem_st_32x32b_x32(t_lane + kQAccCols + slot * kQSlotCols + 32, v1);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_on_leader(&afull[stage], crank);
+      if (lane == 0) arrive_on_leader(&afull[slot], crank);
     }
   exp_done:;
   } else {
