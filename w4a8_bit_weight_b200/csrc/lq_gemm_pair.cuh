@@ -21,18 +21,19 @@
 // the epilogue warps of both CTAs hand it back as soon as it sits in their
 // registers as packed bf16, before any global store.
 //
-// Hand-offs between the two CTAs:
-//   activations landed (odd) -> forwarded to the even CTA's xpeer[stage]
-//   expansion done            -> arrive on the even CTA's afull[slot] (remote for odd)
-//   stage consumed            -> tcgen05.commit multicast to xempty/aempty of both CTAs
-//   tile finished             -> tcgen05.commit multicast to accfull of both CTAs
-//   accumulator loaded        -> arrive on the even CTA's accempty (remote for odd)
+// Activation stage i and TMEM weight slot i are filled and drained together,
+// so one barrier pair covers both.  Hand-offs between the two CTAs:
+//   activations landed   -> both CTAs' activation copies complete their bytes on
+//                           the even CTA's full[stage] (the pair form of TMA)
+//   expansion done       -> arrive on the even CTA's full[stage] (remote for odd)
+//   stage consumed       -> tcgen05.commit multicast to empty[stage] of both CTAs
+//   tile finished        -> tcgen05.commit multicast to accfull of both CTAs
+//   accumulator loaded   -> arrive on the even CTA's accempty (remote for odd)
 // No TMA load uses cluster multicast: each CTA loads its own data.
 //
 // Warp roles (608 threads):
 //   warp 0        TMA producer of weight stages
-//   warp 1        TMEM allocation (both CTAs); MMA issue (even CTA);
-//                 activation-ready forwarding (odd CTA)
+//   warp 1        TMEM allocation (both CTAs); MMA issue (even CTA)
 //   warps 2-9     expansion: two groups of four warps, alternate K-blocks
 //   warps 10-17   epilogue: two warps per TMEM lane quarter, 128 tokens each
 //   warp 18       TMA producer of activation stages
@@ -50,7 +51,7 @@ constexpr int kQBN = 256;                     // weight rows per tile (MMA M, 12
 constexpr int kQBK = 256;                     // K per stage
 constexpr int kQXStages = 4;                  // activation ring
 constexpr int kQWStages = 5;                  // weight ring
-constexpr int kQSlots = 4;                    // TMEM A slots
+constexpr int kQSlots = kQXStages;            // TMEM A slots, paired with activation stages
 constexpr int kQExpGroups = 2;
 constexpr int kQEpiWarp0 = 2 + 4 * kQExpGroups;
 constexpr int kQXProdWarp = kQEpiWarp0 + 8;
@@ -60,7 +61,7 @@ constexpr int kQXBytes = 2 * kQXSub;          // 32 KB: this CTA's 128 tokens x 
 constexpr int kQWBytes = 128 * kQBK / 2;      // 16 KB: 128 rows x 256 codes, 128-byte rows (SW128)
 constexpr int kQSABytes = (kQBK / 64) * 128;  // 4 groups x 128 rows
 constexpr int kQWStage = kQWBytes + 2 * kQSABytes;  // 17 KB, keeps the 1024-byte alignment
-constexpr uint32_t kQTxX = kQXBytes;
+constexpr uint32_t kQTxX = 2 * kQXBytes;      // both CTAs' activations land on the even CTA's barrier
 constexpr uint32_t kQTxW = kQWStage;
 constexpr int kQAccCols = kQBT;               // one accumulator
 constexpr int kQSlotCols = kQBK / 4;          // 64 TMEM columns per expanded stage
@@ -115,6 +116,18 @@ __device__ __forceinline__ void arrive_on_leader(uint64_t* bar, uint32_t crank) 
     mbar_arrive_remote(mapa_shared(smem_u32(bar), 0));
 }
 
+// Tensor load into this CTA's shared memory whose completed bytes are counted
+// on an mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster
+// address, e.g. from mapa).  Plain (non-multicast) copy.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1, uint64_t cache_hint) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(cache_hint)
+      : "memory");
+}
+
 // One elected lane waits; the decision is shared with the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, bool cluster) {
   bool ok = true;
@@ -127,19 +140,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
     w4a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                           const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
                           const GemmArgs p) {
-  constexpr int SX = kQXStages, SW = kQWStages, A = kQSlots;
+  constexpr int SX = kQXStages, SW = kQWStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xring = smem;                 // SX x [2][128 tokens][128 B], SW128
   uint8_t* wring = smem + kQXRing;       // SW x ([128 rows][128 B] SW128 | s [4][128] | a [4][128])
-  uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + kQXRing + kQWRing);
-  uint64_t* xpeer = xfull + SX;          // even CTA: the odd CTA's activations have landed
-  uint64_t* xempty = xpeer + SX;
-  uint64_t* wfull = xempty + SX;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQXRing + kQWRing);  // [SX], used on the even CTA
+  uint64_t* empty = full + SX;           // [SX]
+  uint64_t* wfull = empty + SX;
   uint64_t* wempty = wfull + SW;
-  uint64_t* afull = wempty + SW;         // [A]
-  uint64_t* aempty = afull + A;          // [A]
-  uint64_t* accfull = aempty + A;
+  uint64_t* accfull = wempty + SW;
   uint64_t* accempty = accfull + 1;
   uint64_t* drain = accempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -153,17 +163,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) {
-      mbar_init(&xfull[s], 1);
-      mbar_init(&xpeer[s], 1);
-      mbar_init(&xempty[s], 1);
+      mbar_init(&full[s], 1 + 8);  // even producer's expect-tx + four expansion warps of each CTA
+      mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < SW; ++s) {
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], 4);  // the four warps of the expansion group that read it
-    }
-    for (int s = 0; s < A; ++s) {
-      mbar_init(&afull[s], 8);   // four expansion warps of each CTA
-      mbar_init(&aempty[s], 1);
     }
     mbar_init(accfull, 1);
     mbar_init(accempty, 16);     // eight epilogue warps of each CTA
@@ -233,32 +238,34 @@ __global__ void __launch_bounds__(kQThreads, 1)
     uint64_t pol = 0;
     if (leader) pol = l2_policy_evict_last();
     griddep_wait();  // activations may be the output of the preceding kernel
-    uint32_t issued = 0, issued_par = 0;
+    const uint32_t full_even = mapa_shared(smem_u32(full), 0);
+    bool issued = false;
     int it = 0;
     for (int tile = cid; tile < tiles; tile += ncl) {
       const int xrow = (tile % tiles_m) * kQBT + (int)crank * 128;
       for (int kb = 0; kb < KS; ++kb, ++it) {
         const int x = it % SX;
         const uint32_t use = (uint32_t)(it / SX);
-        if (it >= SX && !warp_wait(&xempty[x], (use & 1u) ^ 1u, abort_flag, false)) goto xprod_done;
+        if (it >= SX && !warp_wait(&empty[x], (use & 1u) ^ 1u, abort_flag, false)) goto xprod_done;
         if (leader) {
           uint8_t* xb = xring + x * kQXBytes;
-          mbar_arrive_expect_tx(&xfull[x], kQTxX);
-          tma_load_2d(xb, &tm_x, &xfull[x], kb * kQBK, xrow, pol);
-          tma_load_2d(xb + kQXSub, &tm_x, &xfull[x], kb * kQBK + 128, xrow, pol);
+          const uint32_t bar = full_even + (uint32_t)(x * 8);
+          if (even) mbar_arrive_expect_tx(&full[x], kQTxX);
+          tma_load_2d_pair(xb, &tm_x, bar, kb * kQBK, xrow, pol);
+          tma_load_2d_pair(xb + kQXSub, &tm_x, bar, kb * kQBK + 128, xrow, pol);
         }
-        issued |= 1u << x;
-        issued_par = (issued_par & ~(1u << x)) | ((use & 1u) << x);
+        issued = true;
       }
     }
   xprod_done:
-    if (leader && *abort_flag)
-      for (int s = 0; s < SX; ++s)
-        if (issued & (1u << s)) {
-          const unsigned long long t0w = globaltimer();
-          while (!mbar_try_wait(smem_u32(&xfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
-          }
-        }
+    // The copies complete on the even CTA's barrier, whose phase also needs the
+    // expansion warps: after an abort, give any copy in flight a fixed 200 us
+    // to land before this CTA's shared memory is released.
+    if (leader && issued && *abort_flag) {
+      const unsigned long long t0w = globaltimer();
+      while (globaltimer() - t0w < 200000ull) {
+      }
+    }
   } else if (warp == 1) {
     if (even) {
       // ------------------------------------------------- MMA issuer (even CTA)
@@ -270,24 +277,18 @@ __global__ void __launch_bounds__(kQThreads, 1)
         if (!warp_wait(accempty, ((uint32_t)j & 1u) ^ 1u, abort_flag, true)) goto mma_done;
         tc_fence_after();
         for (int kb = 0; kb < KS; ++kb, ++it) {
-          const int x = it % SX, slot = it % A;
-          const uint32_t xpar = (uint32_t)(it / SX) & 1u, apar = (uint32_t)(it / A) & 1u;
-          bool ok = true;
-          if (leader)
-            ok = mbar_wait_cluster(&afull[slot], apar, abort_flag) && mbar_wait(&xfull[x], xpar, abort_flag) &&
-                 mbar_wait_cluster(&xpeer[x], xpar, abort_flag);
-          if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) goto mma_done;
+          const int x = it % SX;
+          if (!warp_wait(&full[x], (uint32_t)(it / SX) & 1u, abort_flag, true)) goto mma_done;
           if (leader) {
             tc_fence_after();
             const uint32_t xs = smem_u32(xring + x * kQXBytes);
-            const uint32_t a_col = tmem_base + kQAccCols + slot * kQSlotCols;
+            const uint32_t a_col = tmem_base + kQAccCols + x * kQSlotCols;
 #pragma unroll
             for (int jj = 0; jj < kQBK / 32; ++jj) {
               const uint64_t bdesc = smem_desc_k_sw128(xs + (jj >> 2) * kQXSub) + (uint64_t)(2 * (jj & 3));
               mma_i8_ts_pair(tmem_base, a_col + jj * 8, bdesc, idesc, (kb > 0 || jj > 0) ? 1u : 0u);
             }
-            tc_commit_pair_mc(&xempty[x], 0x3);
-            tc_commit_pair_mc(&aempty[slot], 0x3);
+            tc_commit_pair_mc(&empty[x], 0x3);
           }
           any = true;
         }
@@ -303,14 +304,6 @@ __global__ void __launch_bounds__(kQThreads, 1)
         while (!mbar_try_wait(a, 0) && globaltimer() - t0w < 100000000ull) {
         }
       }
-    } else {
-      // -------------------------- odd CTA: forward "activations landed" to the even CTA
-      const uint32_t peer_xpeer = mapa_shared(smem_u32(xpeer), 0);
-      for (int it = 0; it < total; ++it) {
-        const int x = it % SX;
-        if (!warp_wait(&xfull[x], (uint32_t)(it / SX) & 1u, abort_flag, false)) break;
-        if (leader) mbar_arrive_remote(peer_xpeer + (uint32_t)(x * 8));
-      }
     }
   } else if (warp < kQEpiWarp0) {
     // ------------------------------------------------------ expansion warps
@@ -320,9 +313,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     const int sw = r & 7;                // 128-byte swizzle of this row's 16-byte chunks
     for (int it = grp; it < total; it += kQExpGroups) {
-      const int w = it % SW, slot = it % A;
+      const int w = it % SW, slot = it % SX;
       if (!__all_sync(0xffffffffu, mbar_wait(&wfull[w], (uint32_t)(it / SW) & 1u, abort_flag) &&
-                                       mbar_wait(&aempty[slot], ((uint32_t)(it / A) & 1u) ^ 1u, abort_flag)))
+                                       mbar_wait(&empty[slot], ((uint32_t)(it / SX) & 1u) ^ 1u, abort_flag)))
         goto exp_done;
       tc_fence_after();
       const uint8_t* wb = wring + w * kQWStage;
@@ -354,7 +347,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_on_leader(&afull[slot], crank);
+      if (lane == 0) arrive_on_leader(&full[slot], crank);
     }
   exp_done:;
   } else {
@@ -366,13 +359,20 @@ __global__ void __launch_bounds__(kQThreads, 1)
     griddep_wait();
     int j = 0;
     for (int tile = cid; tile < tiles; tile += ncl, ++j) {
-      if (!warp_wait(accfull, (uint32_t)j & 1u, abort_flag, false)) goto epi_done;
-      tc_fence_after();
       const int tm = tile % tiles_m, tn = tile / tiles_m;
       const int n = tn * kQBN + (int)crank * 128 + r;
       const bool n_ok = n < p.N;
-      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
       const int mb = tm * kQBT + e * 128;
+      // scales are loaded before the accumulator is ready, off the hand-back path
+      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
+      float sx4[4];  // s_x of tokens mb + 32c + lane
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int m = mb + 32 * c + lane;
+        sx4[c] = (!OUT_I32 && m < p.M) ? __ldg(p.s_x + m) : 0.0f;
+      }
+      if (!warp_wait(accfull, (uint32_t)j & 1u, abort_flag, false)) goto epi_done;
+      tc_fence_after();
       if constexpr (OUT_I32) {
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -398,8 +398,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t v[16];
           tmem_ld_32x32b_x16(t_lane + e * 128 + cc * 16, v);
-          const int m = mb + (cc >> 1) * 32 + lane;
-          const float sxl = (m < p.M) ? __ldg(p.s_x + m) : 0.0f;
+          const float sxl = sx4[cc >> 1];
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
