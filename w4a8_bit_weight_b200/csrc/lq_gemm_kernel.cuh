@@ -33,10 +33,11 @@
 // Integer sums are order-independent, so every schedule gives bit-identical
 // results.
 //
-// Programmatic dependent launch: the producer issues the weight loads of the
-// first stages before griddepcontrol.wait (weights are never written by the
-// kernel this launch overlaps), and the activation loads after it; the
-// epilogue waits before it reads scales or writes the output.
+// Programmatic dependent launch: every CTA lets the next kernel launch as soon
+// as its prologue is done; the producer issues the weight loads of the first
+// stages before griddepcontrol.wait (weights are never written by the kernel
+// this launch overlaps), and the activation loads after it; the epilogue
+// waits before it reads scales or writes the output.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -71,7 +72,14 @@ struct GemmCfg {
   static constexpr int kSlots = BT <= 64 ? (kStages < (256 - kAccCols) / 32 ? kStages : (256 - kAccCols) / 32)
                                          : kStages;
   static constexpr int kTmemCols = (kAccCols + kSlots * 32 <= 256) ? 256 : 512;
-  static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * BT * kBlockN * 4 : 0;  // DSMEM partials
+  // Cluster split-K is a reduce-scatter: the tile's 128 x BT partial sums are cut
+  // into CS pieces (row quarters, and token slices of them when CS = 8); each
+  // CTA owns one piece (CS = 2: two quarters) and receives it from the others.
+  static constexpr int kSlices = CS >= 4 ? CS / 4 : 1;            // token slices per row quarter
+  static constexpr int kPieceT = BT / kSlices;                    // tokens per piece
+  static constexpr int kOwned = CS >= 4 ? 1 : (CS == 2 ? 2 : 4);  // pieces (quarters) owned per CTA
+  static constexpr int kPieceBytes = kPieceT * 32 * 4;            // [tokens][32 rows] int32
+  static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * kOwned * kPieceBytes : 0;  // received pieces
   static constexpr int kXRing = kStages * kXBytes;
   static constexpr int kWRing = kStages * kWStage;
   static constexpr int kBarBytes = 512;
@@ -83,7 +91,7 @@ struct GemmCfg {
   static_assert(kAccCols + kSlots * 32 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kXBytes % 1024 == 0 && (kXRing + kWRing + kRedBytes) % 8 == 0, "alignment");
-  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 5 * 8 + 16 <= kBarBytes, "barrier area");
+  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 6 * 8 + 16 <= kBarBytes, "barrier area");
 };
 
 struct GemmArgs {
@@ -95,6 +103,27 @@ struct GemmArgs {
   int M, N, K;
   int tiles_m, KB;
   long long U;           // units = tiles * KB
+};
+
+// (tile, K-block) of a unit, stepped without divisions: an integer division
+// costs a few hundred cycles, as much as the copy it would address.
+struct UnitCursor {
+  int kb, tile_m, tile_n;
+  __device__ __forceinline__ UnitCursor(long long u, int KB, int tiles_m) {
+    const int t = (int)(u / KB);
+    kb = (int)(u - (long long)t * KB);
+    tile_n = t / tiles_m;
+    tile_m = t - tile_n * tiles_m;
+  }
+  __device__ __forceinline__ void next(int KB, int tiles_m) {
+    if (++kb == KB) {
+      kb = 0;
+      if (++tile_m == tiles_m) {
+        tile_m = 0;
+        ++tile_n;
+      }
+    }
+  }
 };
 
 __device__ __forceinline__ long long cta_of_unit(long long u, long long U, long long G) {
@@ -117,6 +146,17 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volat
   const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase, abort_flag));
   phase ^= 1u;
   return ok;
+}
+
+// Output element from an accumulator and the token's scale s_x[m] (given).
+template <bool OUT_I32>
+__device__ __forceinline__ void store_out_sx(const GemmArgs& p, int m, int n, int32_t acc, float sx, float sc) {
+  if constexpr (OUT_I32) {
+    reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = acc;
+  } else {
+    const float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(sx, sc));
+    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
+  }
 }
 
 template <bool OUT_I32>
@@ -145,8 +185,10 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&v)[32]
   }
 }
 
+// CTAs that keep to 256 TMEM columns are meant to share an SM with a CTA of
+// the next launch (programmatic dependent launch): registers are capped for two.
 template <int BT, int CS, bool OUT_I32>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 256 ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
                      const GemmArgs p) {
@@ -168,7 +210,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* drain = accfull + 1;
   uint64_t* grp = drain + 1;
   uint64_t* redbar = grp + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + 1);
+  uint64_t* xfirst = redbar + 1;  // the activation tiles of the first min(S, total) K-blocks, all at once
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xfirst + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -189,7 +232,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     mbar_init(accfull, 1);
     mbar_init(drain, 1);
     mbar_init(grp, 4);
-    mbar_init(redbar, CS >= 2 ? (CS - 1) * 128 : 1);
+    // every CTA of a split-K cluster expects its piece from each of the others
+    mbar_init(redbar, 1);
+    if (CS >= 2) mbar_arrive_expect_tx(redbar, (uint32_t)C::kRedBytes);
+    mbar_init(xfirst, 1);
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -206,6 +252,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The next kernel in the stream may launch now: its griddepcontrol.wait still
+  // waits for this grid to complete, and meanwhile its CTAs, where they fit
+  // beside this one, stream their weights.
+  griddep_launch_dependents();
   // Cluster barrier, first half: this CTA's barriers are initialized.  The
   // second half is waited on only before a remote arrive (and at teardown).
   if constexpr (CS >= 2) cluster_arrive();
@@ -242,40 +292,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     const int total = (int)(u_end - u_begin);
     const int P = min(S, total);
-    if (leader) {
-      // first P K-blocks (they may span tiles in the stream-K schedule)
-      long long u = u_begin;
-      for (int i = 0; i < P; ++i, ++u) {
-        const int t = (int)(u / KB), kb = (int)(u % KB);
-        const int tile_n = t / p.tiles_m;
+    const UnitCursor first(u_begin, KB, p.tiles_m);
+    UnitCursor cw = first;  // after the prefetch: the unit of K-block P (every lane steps it)
+    // first P K-blocks (they may span tiles in the stream-K schedule)
+    for (int i = 0; i < P; ++i, cw.next(KB, p.tiles_m)) {
+      if (leader) {
         uint8_t* wb = wring + i * C::kWStage;
         mbar_arrive_expect_tx(&wfull[i], C::kTxW);
-        tma_load_2d(wb, &tm_w, &wfull[i], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
-        tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], tile_n * kBlockN, kb * 2, pol_stream);
-        tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], tile_n * kBlockN, kb * 2, pol_stream);
+        tma_load_2d(wb, &tm_w, &wfull[i], cw.kb * (kBlockK / 2), cw.tile_n * kBlockN, pol_stream);
+        tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], cw.tile_n * kBlockN, cw.kb * 2, pol_stream);
+        tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], cw.tile_n * kBlockN, cw.kb * 2, pol_stream);
       }
     }
     griddep_wait();
-    if (leader) {
-      long long u = u_begin;
-      for (int i = 0; i < P; ++i, ++u) {
-        const int t = (int)(u / KB), kb = (int)(u % KB);
-        const int tile_m = t % p.tiles_m;
-        mbar_arrive_expect_tx(&xfull[i], C::kTxX);
-        tma_load_2d(xring + i * C::kXBytes, &tm_x, &xfull[i], kb * kBlockK, tile_m * BT, pol_keep);
-      }
+    if (leader && P > 0) {
+      // one barrier for all of them: the MMA warp waits once
+      mbar_arrive_expect_tx(xfirst, (uint32_t)P * C::kTxX);
+      UnitCursor cx = first;
+      for (int i = 0; i < P; ++i, cx.next(KB, p.tiles_m))
+        tma_load_2d(xring + i * C::kXBytes, &tm_x, xfirst, cx.kb * kBlockK, cx.tile_m * BT, pol_keep);
     }
     __syncwarp();
-    uint32_t issued = P >= 32 ? 0xffffffffu : ((1u << P) - 1u), issued_par = 0;
+    // xfull[s] serves the refills of stage s only: its k-th phase is the (k+1)-th use of the stage
+    uint32_t issued = 0, issued_par = 0;
     {
       int stage = P % S;
       uint32_t phase = (uint32_t)(P / S) & 1u;
-      long long u = u_begin + P;
-      for (int it = P; it < total; ++it, ++u) {
+      for (int it = P; it < total; ++it, cw.next(KB, p.tiles_m)) {
         if (!lane0_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
         if (leader) {
-          const int t = (int)(u / KB), kb = (int)(u % KB);
-          const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
+          const int kb = cw.kb, tile_m = cw.tile_m, tile_n = cw.tile_n;
           uint8_t* wb = wring + stage * C::kWStage;
           mbar_arrive_expect_tx(&wfull[stage], C::kTxW);
           tma_load_2d(wb, &tm_w, &wfull[stage], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
@@ -285,7 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(xring + stage * C::kXBytes, &tm_x, &xfull[stage], kb * kBlockK, tile_m * BT, pol_keep);
         }
         issued |= 1u << stage;
-        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        issued_par = (issued_par & ~(1u << stage)) | ((phase ^ 1u) << stage);
         if (++stage == S) {
           stage = 0;
           phase ^= 1u;
@@ -295,54 +341,84 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   producer_done:
     if (leader && *abort_flag) {
       // never leave a bulk copy in flight into shared memory that is about to be released
-      for (int s = 0; s < S; ++s)
-        if (issued & (1u << s)) {
-          const unsigned long long t0w = globaltimer();
-          while (!mbar_try_wait(smem_u32(&wfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
+      const unsigned long long t0w = globaltimer();
+      if (P > 0)
+        while (!mbar_try_wait(smem_u32(xfirst), 0) && globaltimer() - t0w < 100000000ull) {
+        }
+      for (int s = 0; s < S; ++s) {
+        // the last weight load into stage s: use (issued ? refill : first)
+        if (s < P)
+          while (!mbar_try_wait(smem_u32(&wfull[s]), ((issued >> s) & 1u) ? (((issued_par >> s) & 1u) ^ 1u) : 0u) &&
+                 globaltimer() - t0w < 100000000ull) {
           }
+        if (issued & (1u << s))
           while (!mbar_try_wait(smem_u32(&xfull[s]), (issued_par >> s) & 1u) && globaltimer() - t0w < 100000000ull) {
           }
-        }
+      }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = idesc_i8(BT);
-    bool any = false;
-    int stage = 0, slot = 0;
-    uint32_t sphase = 0, aphase = 0;
+    // A wait costs about as much as a K-block of small MMAs, so the loop waits
+    // as little as it can: once for all the preloaded activation tiles; on the
+    // weight side, expansion finishes K-blocks in order, so a completed later
+    // block covers every block before it.  Stages and slots are released only
+    // when a later K-block will reuse them.
+    const int total = (int)(u_end - u_begin);
+    const int P = min(S, total);
+    bool any = false, x_first_seen = false;
+    int it = 0, ready = 0;  // K-blocks [0, ready) are known to be expanded
     for (long long u = u_begin; u < u_end;) {
       const int kb0 = (int)(u % KB);
       const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1;) {
         bool ok = true;
-        if (leader) ok = mbar_wait(&afull[slot], aphase, abort_flag) && mbar_wait(&xfull[stage], sphase, abort_flag);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) goto mma_done;
+        int run = 1;  // K-blocks from `it` on that need no further wait
         if (leader) {
+          const int stage = it % S, slot = it % A;
+          if (it < P) {
+            if (!x_first_seen) ok = mbar_wait(xfirst, 0, abort_flag);
+            x_first_seen = true;
+          } else {
+            ok = mbar_wait(&xfull[stage], (uint32_t)(it / S - 1) & 1u, abort_flag);
+          }
+          if (ok && it >= ready) {
+            ok = mbar_wait(&afull[slot], (uint32_t)(it / A) & 1u, abort_flag);
+            ready = it + 1;
+            // inside the window of preloaded stages the expansion usually runs
+            // ahead (it works while this kernel waits for its inputs): one look
+            // at the furthest block there may cover all the blocks before it
+            const int hi = min(it + A - 1, P - 1);
+            if (ok && hi > it && mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u)) ready = hi + 1;
+          }
+          run = min(min(ready, it < P ? P : it + 1) - it, kb1 - kb);
+        }
+        run = __shfl_sync(0xffffffffu, ok ? run : 0, 0);
+        if (run <= 0) goto mma_done;
+        if (leader) {
+          // the whole run back to back, one thread, no warp synchronization
           tc_fence_after();
-          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
-          const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
+          int stage = it % S, slot = it % A;
+          for (int r = 0; r < run; ++r) {
+            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
+            const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
 #pragma unroll
-          for (int j = 0; j < kBlockK / 32; ++j)
-            mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb > kb0 || j > 0) ? 1u : 0u);
-          tc_commit(&empty[stage]);
-          tc_commit(&aempty[slot]);
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb + r > kb0 || j > 0) ? 1u : 0u);
+            if (it + r + S < total) tc_commit(&empty[stage]);
+            if (it + r + A < total) tc_commit(&aempty[slot]);
+            if (++stage == S) stage = 0;
+            if (++slot == A) slot = 0;
+          }
         }
+        it += run;
+        kb += run;
         any = true;
-        if (++stage == S) {
-          stage = 0;
-          sphase ^= 1u;
-        }
-        if (++slot == A) {
-          slot = 0;
-          aphase ^= 1u;
-        }
       }
       if (leader) tc_commit(accfull);
       __syncwarp();
       u += kb1 - kb0;
     }
-    // the next kernel in the stream may start its prologue
-    griddep_launch_dependents();
   mma_done:
     if (leader && any) {
       // all issued MMAs have finished before TMEM is released
@@ -360,7 +436,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int sw = (r >> 1) & 3;        // 64-byte swizzle of this row's 16-byte chunks
     uint32_t acc_phase = 0, grp_phase = 0;
     bool waited_dep = false;
-    bool red_done = (CS < 2 || crank != 0);
+    // split-K: the warps that own a piece must see all of it arrive before the
+    // CTA may leave (the others' bulk copies write into this CTA)
+    bool red_done = !(CS >= 2 && (CS >= 4 ? sub == (int)crank / C::kSlices : sub / C::kOwned == (int)crank));
     int stage = 0, slot = 0;
     uint32_t sphase = 0, aphase = 0;
     for (long long u = u_begin; u < u_end;) {
@@ -411,64 +489,125 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         griddep_wait();  // scales and the output may belong to the preceding kernel
         waited_dep = true;
       }
+      // scales of this tile, loaded before the accumulator is ready: s_c of this
+      // thread's row, s_x of token m0 + lane of the first column chunk
+      const int n = tile_n * kBlockN + r;
+      const int m0 = tile_m * BT;
+      const bool n_ok = n < p.N;
+      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
+      // the first token this warp writes: split-K clusters write only their own piece
+      constexpr int SXC = CS >= 2 ? (C::kPieceT < 32 ? C::kPieceT : 32) : CH;
+      const int sx0 = m0 + (CS >= 4 ? (int)(crank % C::kSlices) * C::kPieceT : 0);
+      float sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
       acc_phase ^= 1u;
       tc_fence_after();
       {
-        const int n = tile_n * kBlockN + r;
-        const int m0 = tile_m * BT;
-        const bool n_ok = n < p.N;
-        const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
         const bool whole = (kb0 == 0 && kb1 == KB);
         if constexpr (CS >= 2) {
-          // ----------------------------------------- cluster split-K (DSMEM)
-          if (crank != 0) {
-            // the leader's barrier is initialized once the whole cluster has arrived
-            cluster_wait();
-            cl_waited = true;
-            // partial sums -> leader's shared memory, then one release-arrive per thread
-            const uint32_t dst = mapa_shared(smem_u32(red + (size_t)(crank - 1) * BT * kBlockN + r), 0);
+          // ------------------------------ cluster split-K: reduce-scatter (DSMEM)
+          constexpr int T = C::kPieceT;
+          constexpr int TC = T < 32 ? T : 32;  // TMEM columns per load
+          const int q = sub;                   // this warp's row quarter
+          // the other CTAs' barriers are initialized once the whole cluster has arrived
+          cluster_wait();
+          cl_waited = true;
+          // 1. pieces owned by other CTAs: TMEM -> this warp's staging rows
+          //    [token][lane] (in the free activation ring) -> one bulk copy each
+          uint32_t* stg = reinterpret_cast<uint32_t*>(xring) + (size_t)q * BT * 32;
+          bool sent = false;
 #pragma unroll 1
-            for (int cc = 0; cc < BT / CH; ++cc) {
+          for (int h = 0; h < C::kSlices; ++h) {
+            const int o = CS >= 4 ? q * C::kSlices + h : q / C::kOwned;
+            if (o == (int)crank) continue;
+#pragma unroll 1
+            for (int c = 0; c < T / TC; ++c) {
               uint32_t v[32];
-              tmem_load_cols<CH>(t_lane + cc * CH, v);
+              const uint32_t col = (uint32_t)(h * T + c * TC);
+              if constexpr (TC == 8) {
+                uint32_t v8[8];
+                tmem_ld_32x32b_x8(t_lane + col, v8);
+                tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < CH; ++i) st_cluster_u32(dst + (uint32_t)((cc * CH + i) * kBlockN * 4), v[i]);
+                for (int i = 0; i < 8; ++i) v[i] = v8[i];
+              } else {
+                tmem_load_cols<TC>(t_lane + col, v);
+              }
+#pragma unroll
+              for (int i = 0; i < TC; ++i) stg[(col + i) * 32 + lane] = v[i];
             }
-            tc_fence_before();
-            mbar_arrive_remote(mapa_shared(smem_u32(redbar), 0));
-          } else {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const int slot = (int)crank < o ? (int)crank : (int)crank - 1;
+              const int pidx = CS >= 4 ? 0 : q % C::kOwned;
+              const uint32_t dst = mapa_shared(smem_u32(red + ((size_t)slot * C::kOwned + pidx) * T * 32), (uint32_t)o);
+              bulk_copy_s2s(dst, stg + (size_t)h * T * 32, (uint32_t)C::kPieceBytes, mapa_shared(smem_u32(redbar), (uint32_t)o));
+              bulk_commit();
+            }
+            sent = true;
+          }
+          // 2. the piece this warp owns, if any: own partial + the others' pieces
+#pragma unroll 1
+          for (int h = 0; h < C::kSlices; ++h) {
+            const int o = CS >= 4 ? q * C::kSlices + h : q / C::kOwned;
+            if (o != (int)crank) continue;
+            // every lane observes the completed bytes itself (cluster-scope acquire)
             if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
             red_done = true;
+            const int pidx = CS >= 4 ? 0 : q % C::kOwned;
 #pragma unroll 1
-            for (int cc = 0; cc < BT / CH; ++cc) {
+            for (int c = 0; c < T / TC; ++c) {
+              const float sx_cur = sx_next;
+              if (c + 1 < T / TC) {
+                const int mn = m0 + h * T + (c + 1) * TC + lane;
+                sx_next = (!OUT_I32 && lane < TC && mn < p.M) ? __ldg(p.s_x + mn) : 0.0f;
+              }
               uint32_t v[32];
-              tmem_load_cols<CH>(t_lane + cc * CH, v);
+              const uint32_t col = (uint32_t)(h * T + c * TC);
+              if constexpr (TC == 8) {
+                uint32_t v8[8];
+                tmem_ld_32x32b_x8(t_lane + col, v8);
+                tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < CH; ++i) {
-                const int ml = cc * CH + i;
-                int32_t acc = (int32_t)v[i];
+                for (int i = 0; i < 8; ++i) v[i] = v8[i];
+              } else {
+                tmem_load_cols<TC>(t_lane + col, v);
+              }
+#pragma unroll 1
+              for (int sidx = 0; sidx < CS - 1; ++sidx) {
+                const int32_t* rp = red + ((size_t)sidx * C::kOwned + pidx) * T * 32 + (size_t)c * TC * 32 + lane;
 #pragma unroll
-                for (int j = 0; j < CS - 1; ++j) acc += red[((size_t)j * BT + ml) * kBlockN + r];
-                const int m = m0 + ml;
-                if (m < p.M && n_ok) store_out<OUT_I32>(p, m, n, acc, sc);
+                for (int i = 0; i < TC; ++i) v[i] += (uint32_t)rp[i * 32];
+              }
+#pragma unroll
+              for (int i = 0; i < TC; ++i) {
+                const int m = m0 + h * T + c * TC + i;
+                const float sx = __shfl_sync(0xffffffffu, sx_cur, i);
+                if (m < p.M && n_ok) store_out_sx<OUT_I32>(p, m, n, (int32_t)v[i], sx, sc);
               }
             }
-            tc_fence_before();
           }
+          tc_fence_before();
+          // the staging rows are read by the bulk copies before this CTA may leave
+          if (sent && lane == 0) bulk_wait_read();
         } else {
           int32_t* ws_tile = p.ws + (size_t)t * BT * kBlockN;
 #pragma unroll 1
           for (int cc = 0; cc < BT / CH; ++cc) {
+            const float sx_cur = sx_next;
+            if (cc + 1 < BT / CH)
+              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < p.M) ? __ldg(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
             uint32_t v[32];
             tmem_load_cols<CH>(t_lane + cc * CH, v);
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
               const int ml = cc * CH + i;
               const int m = m0 + ml;
+              const float sx = __shfl_sync(0xffffffffu, sx_cur, i);
               if (m < p.M) {
                 if (whole) {
-                  if (n_ok) store_out<OUT_I32>(p, m, n, (int32_t)v[i], sc);
+                  if (n_ok) store_out_sx<OUT_I32>(p, m, n, (int32_t)v[i], sx, sc);
                 } else {
                   atomicAdd(ws_tile + ml * kBlockN + r, (int32_t)v[i]);
                 }
@@ -512,9 +651,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       u += kb1 - kb0;
     }
   epi_done:
+    // no bulk copy may still be reading this CTA's staging rows when it leaves
+    if (CS >= 2 && lane == 0) bulk_wait_read();
     if (!red_done) {
-      // leader on an error path: non-leaders may still be writing into this
-      // CTA's shared memory; wait (bounded) for their arrivals before leaving
+      // owner on an error path: the other CTAs may still be copying into this
+      // CTA's shared memory; wait (bounded) for their bytes before leaving
       const uint32_t a = smem_u32(redbar);
       const unsigned long long t0w = globaltimer();
       while (!mbar_try_wait_cluster(a, 0) && globaltimer() - t0w < 100000000ull) {
