@@ -248,7 +248,7 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream(dev)
     counter = [0]
 
-    def step(events=None, e2e=False):
+    def step(e2e=False):
         for M in Ms:
             if e2e:
                 Xd_e2e[:M].copy_(X_host[:M], non_blocking=True)
@@ -258,23 +258,23 @@ def run_ours(args, rank, world, local_rank):
             lq.lq_quantize_act(src, out=(xq_buf[M], sx_buf[M]))
             wq = sets[counter[0] % n_sets]
             counter[0] += 1
-            if events is not None:
-                e0 = torch.cuda.Event(enable_timing=True, external=True)
-                e1 = torch.cuda.Event(enable_timing=True, external=True)
-                e0.record()
-                lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=out_buf[M], workspace_buf=ws)
-                e1.record()
-                events.append((M, e0, e1))
-            else:
-                lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=out_buf[M], workspace_buf=ws)
+            lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=out_buf[M], workspace_buf=ws)
             if e2e:
                 out_host[M].copy_(out_buf[M], non_blocking=True)
 
-    def capture(nsteps, events=None, e2e=False):
+    def capture(nsteps, e2e=False):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for _ in range(nsteps):
-                step(events, e2e)
+                step(e2e)
+        return g
+
+    def capture_gemms(M, n):
+        """n back-to-back GEMMs of one M, the weights rotating over the L2-cold copies."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *sets[i % n_sets], out=out_buf[M], workspace_buf=ws)
         return g
 
     with torch.cuda.stream(stream):
@@ -285,10 +285,8 @@ def run_ours(args, rank, world, local_rank):
         st = lq.lq_get_device_error(dev)
         if st != 0:
             raise RuntimeError(f"device error after warm-up: {st}")
-        gemm_events = []
         g_timed = capture(args.steps)
-        g_instr = capture(args.steps, events=gemm_events)
-        g_soak = capture(max(1, min(args.steps, 50)))
+        g_gemm = {M: capture_gemms(M, args.steps) for M in Ms}
         g_e2e = None if args.no_e2e else capture(args.steps, e2e=True)
 
     uuid = None
@@ -299,11 +297,17 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(uuid) if rank == 0 else None
     time.sleep(0.3)
     t_load0 = time.time()
-    # untimed soak so the clocks settle and the sampler sees load
-    soak_end = time.time() + args.soak_s
-    while time.time() < soak_end:
-        g_soak.replay()
+    # Every timed graph is replayed once untimed first (its first launch also
+    # uploads it to the device), then an untimed soak of the step graph so the
+    # clocks settle and the sampler sees load.
+    with torch.cuda.stream(stream):
+        for g in [g_timed, *g_gemm.values()] + ([g_e2e] if g_e2e is not None else []):
+            g.replay()
         torch.cuda.synchronize(dev)
+        soak_end = time.time() + args.soak_s
+        while time.time() < soak_end:
+            g_timed.replay()
+            torch.cuda.synchronize(dev)
 
     def timed(graph):
         if world > 1:
@@ -319,11 +323,10 @@ def run_ours(args, rank, world, local_rank):
 
     with torch.cuda.stream(stream):
         ms_total = timed(g_timed)
-        # the same K steps with CUDA events around every GEMM node: the GEMM's own
-        # duration per launch (events between kernels also cut the launch overlap,
-        # so these durations include each launch's full ramp-up and tail)
-        ms_instr = timed(g_instr)
-        gemm_ms = [(M, a.elapsed_time(b)) for M, a, b in gemm_events]
+        # the dominant kernel on its own: K back-to-back GEMMs per M in one graph
+        # (the launches overlap through programmatic dependent launch as they do
+        # in the step); its duration per launch is the replay time / K
+        gemm_ms = {M: timed(g_gemm[M]) / args.steps for M in Ms}
         ms_e2e = timed(g_e2e) if g_e2e is not None else None
     t_load1 = time.time()
     clocks = sampler.stop(t_load0, t_load1) if sampler else None
@@ -333,15 +336,15 @@ def run_ours(args, rank, world, local_rank):
 
     K_ = args.steps
     value = world * step_bytes * K_ / (ms_total * 1e-3) / 1e9
-    # dominant kernel: the GEMM, averaged over every launch in the timed region
-    per_M = {M: float(np.mean([t for m, t in gemm_ms if m == M])) for M in Ms}
-    gemm_time_s = sum(t for _, t in gemm_ms) * 1e-3
-    gemm_bytes_total = sum(gemm_bytes(M, w.N, w.K) for M, _ in gemm_ms)
+    # dominant kernel: the GEMM, one launch of each M
+    per_M = {M: float(t) for M, t in gemm_ms.items()}
+    gemm_time_s = sum(per_M.values()) * 1e-3
+    gemm_bytes_total = sum(gemm_bytes(M, w.N, w.K) for M in Ms)
     achieved = gemm_bytes_total / gemm_time_s / 1e9
     pk, pk_src = peaks()
     hbm_peak = float(pk["hbm_gbs"])
     int8_peak = INT8_OVER_BF16 * float(pk["bf16_tflops"])
-    gemm_launches = len(gemm_ms)
+    gemm_launches = args.steps * len(Ms)
     n_traffic = ncu_traffic(args.workload)
     res = {
         "metric": "W4A8 GEMM TOPS and HBM GB/s vs roofline at decode M=1-16 and prefill M=4096",
@@ -373,9 +376,9 @@ def run_ours(args, rank, world, local_rank):
             "peak_source": pk_src,
             "per_launch_us": {str(M): 1e3 * t for M, t in per_M.items()},
             "launches": gemm_launches,
-            "how": "CUDA events around every GEMM node of a replay of the same K steps, "
-                   "right after the timed replay",
-            "instrumented_ms_per_step": ms_instr / args.steps,
+            "how": "per M, K back-to-back lq_w4a8_gemm calls (weights rotating over the L2-cold "
+                   "copies) in one CUDA graph between CUDA events, right after the timed step "
+                   "replay; duration per launch = replay time / K",
             "bytes_per_launch": {str(M): gemm_bytes(M, w.N, w.K) for M in Ms},
         },
         "clocks": clocks,
@@ -405,8 +408,8 @@ def run_ours(args, rank, world, local_rank):
 
 def secondary_workload(name, dev, steps=20):
     """A short measurement of another workload in the same run (the metric also names
-    prefill M=4096): K steps of act-quant + GEMM in one CUDA graph, then the GEMM's own
-    duration from events around each GEMM node of a second replay."""
+    prefill M=4096): K steps of act-quant + GEMM in one CUDA graph, then K back-to-back
+    GEMMs in another for the GEMM's own duration per launch."""
     import w4a8_bit_weight_b200 as lq
     from w4a8_bit_weight_b200 import synth
     w = synth.WORKLOADS[name]
@@ -424,21 +427,21 @@ def secondary_workload(name, dev, steps=20):
         sx = torch.empty(M, dtype=torch.float32, device=dev)
         out = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
         cnt = [0]
-        evs = []
 
-        def one(events=None):
-            lq.lq_quantize_act(Xd[:M], out=(xq, sx))
+        def one(quant=True):
+            if quant:
+                lq.lq_quantize_act(Xd[:M], out=(xq, sx))
             wq = sets[cnt[0] % n_sets]
             cnt[0] += 1
-            if events is None:
-                lq.lq_w4a8_gemm(xq, sx, *wq, out=out)
-            else:
-                e0 = torch.cuda.Event(enable_timing=True, external=True)
-                e1 = torch.cuda.Event(enable_timing=True, external=True)
-                e0.record()
-                lq.lq_w4a8_gemm(xq, sx, *wq, out=out)
-                e1.record()
-                events.append((e0, e1))
+            lq.lq_w4a8_gemm(xq, sx, *wq, out=out)
+
+        def time_graph(g):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            return a.elapsed_time(b) / steps
 
         with torch.cuda.stream(stream):
             for _ in range(3):
@@ -451,18 +454,12 @@ def secondary_workload(name, dev, steps=20):
             gi = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gi, stream=stream):
                 for _ in range(steps):
-                    one(evs)
+                    one(quant=False)
             g.replay()
-            torch.cuda.synchronize(dev)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            g.replay()
-            b.record(stream)
-            torch.cuda.synchronize(dev)
-            ms = a.elapsed_time(b) / steps
             gi.replay()
             torch.cuda.synchronize(dev)
-        gemm_ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+            ms = time_graph(g)
+            gemm_ms = time_graph(gi)
         ops = 2.0 * M * w.N * w.K
         res[str(M)] = {"ms_per_step": ms, "tops_step": ops / (ms * 1e-3) / 1e12,
                        "gemm_us": 1e3 * gemm_ms, "gemm_tops": ops / (gemm_ms * 1e-3) / 1e12,

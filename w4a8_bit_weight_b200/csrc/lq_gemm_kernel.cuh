@@ -148,6 +148,31 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volat
   return ok;
 }
 
+// Writes TC consecutive tokens [m_first, m_first + TC) of this thread's output
+// column n from the accumulators v.  sx_lane holds s_x[m_first + lane] (lanes
+// < TC).  The token scales are gathered first, so that the stores do not wait
+// on one another.  Every lane of the warp must call it.
+template <bool OUT_I32, int TC>
+__device__ __forceinline__ void store_chunk(const GemmArgs& p, int m_first, int n, bool n_ok, const uint32_t* v,
+                                            float sx_lane, float sc) {
+  float scale[TC];
+#pragma unroll
+  for (int i = 0; i < TC; ++i) scale[i] = __fmul_rn(__shfl_sync(0xffffffffu, sx_lane, i), sc);
+  if (!n_ok) return;
+  const int mlim = p.M - m_first;
+  if constexpr (OUT_I32) {
+    int32_t* o = reinterpret_cast<int32_t*>(p.out) + (size_t)m_first * p.N + n;
+#pragma unroll
+    for (int i = 0; i < TC; ++i)
+      if (i < mlim) o[(size_t)i * p.N] = (int32_t)v[i];
+  } else {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m_first * p.N + n;
+#pragma unroll
+    for (int i = 0; i < TC; ++i)
+      if (i < mlim) o[(size_t)i * p.N] = __float2bfloat16_rn(__fmul_rn(__int2float_rn((int32_t)v[i]), scale[i]));
+  }
+}
+
 // Output element from an accumulator and the token's scale s_x[m] (given).
 template <bool OUT_I32>
 __device__ __forceinline__ void store_out_sx(const GemmArgs& p, int m, int n, int32_t acc, float sx, float sc) {
@@ -574,18 +599,13 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
               } else {
                 tmem_load_cols<TC>(t_lane + col, v);
               }
-#pragma unroll 1
+#pragma unroll
               for (int sidx = 0; sidx < CS - 1; ++sidx) {
                 const int32_t* rp = red + ((size_t)sidx * C::kOwned + pidx) * T * 32 + (size_t)c * TC * 32 + lane;
 #pragma unroll
                 for (int i = 0; i < TC; ++i) v[i] += (uint32_t)rp[i * 32];
               }
-#pragma unroll
-              for (int i = 0; i < TC; ++i) {
-                const int m = m0 + h * T + c * TC + i;
-                const float sx = __shfl_sync(0xffffffffu, sx_cur, i);
-                if (m < p.M && n_ok) store_out_sx<OUT_I32>(p, m, n, (int32_t)v[i], sx, sc);
-              }
+              store_chunk<OUT_I32, TC>(p, m0 + h * T + c * TC, n, n_ok, v, sx_cur, sc);
             }
           }
           tc_fence_before();
@@ -600,17 +620,13 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
               sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < p.M) ? __ldg(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
             uint32_t v[32];
             tmem_load_cols<CH>(t_lane + cc * CH, v);
+            if (whole) {
+              store_chunk<OUT_I32, CH>(p, m0 + cc * CH, n, n_ok, v, sx_cur, sc);
+            } else {
 #pragma unroll
-            for (int i = 0; i < CH; ++i) {
-              const int ml = cc * CH + i;
-              const int m = m0 + ml;
-              const float sx = __shfl_sync(0xffffffffu, sx_cur, i);
-              if (m < p.M) {
-                if (whole) {
-                  if (n_ok) store_out_sx<OUT_I32>(p, m, n, (int32_t)v[i], sx, sc);
-                } else {
-                  atomicAdd(ws_tile + ml * kBlockN + r, (int32_t)v[i]);
-                }
+              for (int i = 0; i < CH; ++i) {
+                const int ml = cc * CH + i;
+                if (m0 + ml < p.M) atomicAdd(ws_tile + ml * kBlockN + r, (int32_t)v[i]);
               }
             }
           }
