@@ -70,16 +70,17 @@ def gemm_bytes(M, N, K, G=64):
     return N * K // 2 + 2 * N * (K // G) + 4 * N + M * K + 4 * M + 2 * M * N
 
 
-def actq_bytes(M, K):
-    """bf16 activations in, int8 codes and fp32 scales out."""
-    return 2 * M * K + M * K + 4 * M
+def linear_bytes(M, N, K, G=64):
+    """Algorithmic HBM bytes of one activation-quantization + GEMM pass: the
+    weights, bf16 activations in and bf16 output (the INT8 codes and token scales
+    are intermediates; the fused launch never writes them)."""
+    return N * K // 2 + 2 * N * (K // G) + 4 * N + 2 * M * K + 2 * M * N
 
 
 def step_accounting(w):
-    gb = sum(gemm_bytes(M, w.N, w.K) for M in w.Ms)
-    ab = sum(actq_bytes(M, w.K) for M in w.Ms)
+    gb = sum(linear_bytes(M, w.N, w.K) for M in w.Ms)
     ops = sum(2 * M * w.N * w.K for M in w.Ms)
-    return gb, ab, ops
+    return gb, 0, ops
 
 
 def peaks():
@@ -205,7 +206,7 @@ def cpu_baseline(w, budget_s=10.0):
               f"epilogue) for M in {Ms}" + ("" if frac == 1 else f" with min(M,64) token rows") +
               f", N={w.N}, K={w.K}; {el:.1f} s")
     # throughput in the same unit: the step's algorithmic bytes, scaled to the rows sampled
-    byts = (sum(gemm_bytes(rows[M], w.N, w.K) for M in Ms) + sum(actq_bytes(rows[M], w.K) for M in Ms))
+    byts = sum(linear_bytes(rows[M], w.N, w.K) for M in Ms)
     return {"value": byts * steps / el / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle", "sample": sample,
             "tops": 2 * sum(rows[M] for M in Ms) * w.N * w.K * steps / el / 1e12}
@@ -240,6 +241,9 @@ def run_ours(args, rank, world, local_rank):
     out_buf = {M: torch.empty(M, w.N, dtype=torch.bfloat16, device=dev) for M in Ms}
     ws_need = max(lq.lq_w4a8_gemm_workspace_size(M, w.N, w.K) for M in Ms)
     ws = torch.zeros(max(ws_need, 16), dtype=torch.uint8, device=dev)
+    # lq_w4a8_linear's workspace, for its side measurement (fused vs two launches)
+    lin_ws_need = max(lq.lq_w4a8_linear_workspace_size(M, w.N, w.K, lq.LINEAR_TWO_LAUNCHES) for M in Ms)
+    ws_lin = torch.zeros(max(lin_ws_need, 16), dtype=torch.uint8, device=dev)
     # pinned host buffers for the end-to-end variant
     X_host = X.pin_memory()
     out_host = {M: torch.empty(M, w.N, dtype=torch.bfloat16).pin_memory() for M in Ms}
@@ -277,6 +281,21 @@ def run_ours(args, rank, world, local_rank):
                 lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *sets[i % n_sets], out=out_buf[M], workspace_buf=ws)
         return g
 
+    lin_paths = {"fused": lq.LINEAR_FUSED, "two_launches": lq.LINEAR_TWO_LAUNCHES}
+    n_lin = min(args.steps, 100)
+
+    def capture_linear(M, path):
+        """n_lin back-to-back lq_w4a8_linear calls of one M on one path (None if it does not apply)."""
+        if path == lq.LINEAR_FUSED and lq.lq_w4a8_linear_workspace_size(M, w.N, w.K, path) != 0:
+            return None
+        for i in range(2):
+            lq.lq_w4a8_linear(Xd[:M], *sets[i % n_sets], out=out_buf[M], workspace_buf=ws_lin, path=path)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n_lin):
+                lq.lq_w4a8_linear(Xd[:M], *sets[i % n_sets], out=out_buf[M], workspace_buf=ws_lin, path=path)
+        return g
+
     with torch.cuda.stream(stream):
         # warm-up, eager, W steps (first launches also load the kernels)
         for _ in range(max(args.warmup, 3)):
@@ -287,6 +306,7 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device error after warm-up: {st}")
         g_timed = capture(args.steps)
         g_gemm = {M: capture_gemms(M, args.steps) for M in Ms}
+        g_lin = {} if args.no_secondary else {(M, k): capture_linear(M, p) for M in Ms for k, p in lin_paths.items()}
         g_e2e = None if args.no_e2e else capture(args.steps, e2e=True)
 
     uuid = None
@@ -301,7 +321,8 @@ def run_ours(args, rank, world, local_rank):
     # uploads it to the device), then an untimed soak of the step graph so the
     # clocks settle and the sampler sees load.
     with torch.cuda.stream(stream):
-        for g in [g_timed, *g_gemm.values()] + ([g_e2e] if g_e2e is not None else []):
+        for g in [g_timed, *g_gemm.values(), *[x for x in g_lin.values() if x is not None]] + (
+                [g_e2e] if g_e2e is not None else []):
             g.replay()
         torch.cuda.synchronize(dev)
         soak_end = time.time() + args.soak_s
@@ -328,6 +349,7 @@ def run_ours(args, rank, world, local_rank):
         # in the step); its duration per launch is the replay time / K
         gemm_ms = {M: timed(g_gemm[M]) / args.steps for M in Ms}
         ms_e2e = timed(g_e2e) if g_e2e is not None else None
+        lin_us = {key: (1e3 * timed(g) / n_lin if g is not None else None) for key, g in g_lin.items()}
     t_load1 = time.time()
     clocks = sampler.stop(t_load0, t_load1) if sampler else None
     st = lq.lq_get_device_error(dev)
@@ -391,6 +413,13 @@ def run_ours(args, rank, world, local_rank):
                       "ms_per_step": ms_e2e / K_,
                       "how": "pinned host X -> device copy, quantize_act + gemm, device -> pinned host out, "
                              "per M, same CUDA graph method"}
+    if lin_us:
+        res["linear"] = {
+            "what": "lq_w4a8_linear (activation quantization + GEMM) per M, one fused launch vs the "
+                    "two launches, each as back-to-back calls of one M in one CUDA graph; us per call",
+            **{str(M): {"fused_us": lin_us[(M, "fused")], "two_launches_us": lin_us[(M, "two_launches")],
+                        "auto_path": "fused" if lq.lq_w4a8_linear_workspace_size(M, w.N, w.K) == 0
+                        else "two_launches"} for M in Ms}}
     res["int8_peak_tops"] = int8_peak
     if args.workload == "decode" and not args.no_secondary:
         pre = secondary_workload("prefill", dev)

@@ -180,6 +180,46 @@ LQ_API lq_status lq_w4a8_gemm_ex(const int8_t* x_q, const float* s_x, const uint
                                  int block_t, int schedule, int split_k, int grid, int out_i32,
                                  void* stream);
 
+/* Paths of lq_w4a8_linear_ex. */
+#define LQ_LINEAR_AUTO 0          /* what lq_w4a8_linear uses */
+#define LQ_LINEAR_TWO_LAUNCHES 1  /* lq_quantize_act, then lq_w4a8_gemm */
+#define LQ_LINEAR_FUSED 2         /* one launch; LQ_ERR_UNSUPPORTED_SHAPE where it does not apply */
+
+/*
+ * lq_w4a8_linear -- activation quantization and the GEMM in one call: the
+ * result is bit-identical to lq_quantize_act(X) followed by lq_w4a8_gemm (the
+ * same per-token INT8 codes and s_x, the same contraction and epilogue).
+ *   X_bf16 [M, K] bf16 in, 16-byte aligned; qw, s_u8, a_u8, s_c and out_bf16
+ *   as in lq_w4a8_gemm; same shape rules.
+ *   The fused path applies to decode-sized batches (M <= 16) whose automatic
+ *   schedule is a split-K cluster of 16-token tiles with each CTA's whole
+ *   K-slice in shared memory (e.g. N = K = 4096): ONE launch, in which each
+ *   CTA quantizes its K-slice of X itself and the cluster combines the row
+ *   maxima through distributed shared memory; neither x_q nor s_x is written
+ *   to memory and the workspace size is 0.  lq_w4a8_linear takes it for
+ *   M <= 8 (on B200 at N = K = 4096 it is ahead of the two launches there and
+ *   behind from M = 12, where each quantizing warp has more tokens); the
+ *   other cases are the two launches, with x_q, s_x and the GEMM's workspace
+ *   carved from `workspace`, which must hold
+ *   lq_w4a8_linear_workspace_size(M, N, K) bytes, be 16-byte aligned and
+ *   follow lq_w4a8_gemm's zero-fill rule (else LQ_ERR_WORKSPACE).
+ *   lq_w4a8_linear_ex chooses the path (LQ_LINEAR_*; anything else is
+ *   LQ_ERR_INVALID_ARG); its workspace size is lq_w4a8_linear_workspace_size_ex.
+ *   Launch overlap as for lq_w4a8_gemm: X is read only after the preceding
+ *   kernel in the stream has completed.
+ *   The fused path is this library's (the pages quantize activations as a
+ *   separate step); it changes when the work happens, not what is computed.
+ */
+LQ_API size_t lq_w4a8_linear_workspace_size(int M, int N, int K);
+LQ_API lq_status lq_w4a8_linear(const void* X_bf16, const uint8_t* qw, const uint8_t* s_u8,
+                                const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K,
+                                int group, void* workspace, size_t workspace_bytes, void* stream);
+LQ_API size_t lq_w4a8_linear_workspace_size_ex(int M, int N, int K, int path);
+LQ_API lq_status lq_w4a8_linear_ex(const void* X_bf16, const uint8_t* qw, const uint8_t* s_u8,
+                                   const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N,
+                                   int K, int group, void* workspace, size_t workspace_bytes, int path,
+                                   void* stream);
+
 /*
  * lq_w4a8_gemm_i32 -- the contraction only: acc[m,n] as int32 [M, N] (16-byte
  * aligned), same operands, rules and workspace as lq_w4a8_gemm.

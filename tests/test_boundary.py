@@ -98,3 +98,44 @@ def test_workspace_size_rules(lib):
     assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 3, 0, 2) == 0
     # 3 CTAs over 2 tiles x 4 K-blocks: split tiles need [tiles][16][128] int32 + tickets
     assert lib.lq_w4a8_gemm_workspace_size_ex(16, 256, 512, 16, 3, 0, 3) == 2 * 16 * 128 * 4 + 16
+
+
+def test_linear_rejects_before_launch(lib):
+    f = lib.lq_w4a8_linear
+
+    def call(M=16, N=256, K=512, group=64, X=GOOD, qw=GOOD, s=GOOD, a=GOOD, sc=GOOD, out=GOOD):
+        return f(X, qw, s, a, sc, out, M, N, K, group, None, 0, None)
+
+    assert call(group=32) == 2
+    assert call(K=192) == 2
+    assert call(N=200) == 2
+    assert call(M=-1) == 1
+    assert call(X=P(0)) == 1
+    assert call(sc=P(0)) == 1
+    assert call(out=P(0)) == 1
+    assert call(X=ODD) == 3
+    assert call(out=ODD) == 3
+    assert call(sc=P((1 << 20) + 2)) == 3
+    assert f(None, None, None, None, None, None, 0, 256, 512, 64, None, 0, None) == 0  # empty batch
+    fx = lib.lq_w4a8_linear_ex
+    assert fx(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 16, 256, 512, 64, None, 0, 3, None) == 1   # unknown path
+    assert fx(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 16, 256, 512, 64, None, 0, -1, None) == 1
+
+
+def test_linear_workspace_size_rules(lib):
+    w = lib.lq_w4a8_linear_workspace_size
+    wx = lib.lq_w4a8_linear_workspace_size_ex
+    # small batches in split-K clusters whose CTAs preload their K-slice: one fused launch
+    assert w(1, 4096, 4096) == 0
+    assert w(8, 4096, 4096) == 0
+    assert w(8, 2048, 4096) == 0
+    # 9..16 tokens may take it too, but the automatic path uses two launches there
+    assert wx(16, 4096, 4096, 2) == 0
+    assert w(16, 4096, 4096) == 16 * 4096 + 64
+    assert wx(4, 4096, 4096, 1) == 4 * 4096 + 16
+    # otherwise two launches: x_q and s_x (16-byte aligned) carved from the workspace
+    assert w(24, 4096, 4096) == 24 * 4096 + 96
+    assert w(16, 256, 512) == 16 * 512 + 64
+    assert w(16, 4096, 14336) == 16 * 14336 + 64
+    assert w(16, 200, 512) == 0   # invalid shape
+    assert wx(16, 4096, 4096, 5) == 0  # invalid path

@@ -70,6 +70,10 @@ def load_library(path: str = LIB_PATH):
             "lq_dequant_weights_i8": ([P, P, P, I, I, I, P, P], I),
             "lq_get_device_error": ([P], I),
             "lq_w4a8_gemm_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, P], I),
+            "lq_w4a8_linear_workspace_size": ([I, I, I], Z),
+            "lq_w4a8_linear": ([P, P, P, P, P, P, I, I, I, I, P, Z, P], I),
+            "lq_w4a8_linear_workspace_size_ex": ([I, I, I, I], Z),
+            "lq_w4a8_linear_ex": ([P, P, P, P, P, P, I, I, I, I, P, Z, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -117,11 +121,13 @@ def _need(t: torch.Tensor, dtype, name: str, shape=None):
 _ws = {}
 
 
-def workspace(nbytes: int, device) -> torch.Tensor | None:
+def workspace(nbytes: int, device, kind: str = "gemm") -> torch.Tensor | None:
+    """kind "gemm": the GEMM's zero-filled scratch; kind "linear": lq_w4a8_linear's,
+    whose front holds x_q and s_x (so it is never zero there) -- kept apart."""
     if nbytes == 0:
         return None
     dev = torch.device(device)
-    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    key = (kind, dev.index if dev.index is not None else torch.cuda.current_device())
     buf = _ws.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=dev)
@@ -232,6 +238,42 @@ def lq_w4a8_gemm_i32(x_q, qw, s_u8, a_u8, out=None, group: int = GROUP, block_t:
     """The int32 accumulators x_q @ dequant(qw)^T -> [M, N] int32."""
     return _gemm(x_q, None, qw, s_u8, a_u8, None, out, group, block_t, split_k, grid, True, workspace_buf,
                  schedule)
+
+
+# paths of lq_w4a8_linear (LQ_LINEAR_* in lq.h)
+LINEAR_AUTO, LINEAR_TWO_LAUNCHES, LINEAR_FUSED = 0, 1, 2
+
+
+def lq_w4a8_linear_workspace_size(M: int, N: int, K: int, path: int = LINEAR_AUTO) -> int:
+    return int(load_library().lq_w4a8_linear_workspace_size_ex(M, N, K, path))
+
+
+def lq_w4a8_linear(X, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP, workspace_buf=None,
+                   path: int = LINEAR_AUTO):
+    """Activation quantization + W4A8 GEMM in one call: bf16 X [M, K] -> [M, N] bf16,
+    bit-identical to lq_w4a8_gemm(*lq_quantize_act(X), ...).  One fused launch for
+    small decode batches, two launches otherwise (lq_w4a8_linear in lq.h); `path`
+    forces one of them (LINEAR_*)."""
+    lib = load_library()
+    _need(X, torch.bfloat16, "X")
+    M, K = X.shape
+    N = qw.shape[0]
+    _need(qw, torch.uint8, "qw", (N, K // 2))
+    _need(s_u8, torch.uint8, "s_u8", (K // group, N))
+    _need(a_u8, torch.uint8, "a_u8", (K // group, N))
+    _need(s_c, torch.float32, "s_c", (N,))
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+    _need(out, torch.bfloat16, "out", (M, N))
+    with torch.cuda.device(X.device):
+        ws = workspace_buf
+        if ws is None:
+            ws = workspace(lq_w4a8_linear_workspace_size(M, N, K, path), X.device, kind="linear")
+        nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+        _check("lq_w4a8_linear", lib.lq_w4a8_linear_ex(
+            _ptr(X), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out), M, N, K, group,
+            _ptr(ws), nbytes, path, _stream(X.device)))
+    return out
 
 
 def lq_w4a8_gemm_noalloc(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP):

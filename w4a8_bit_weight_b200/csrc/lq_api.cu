@@ -349,6 +349,7 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return LQ_ERR_CUDA;
   lq::GemmArgs a;
+  a.x_bf16 = nullptr;
   a.s_x = s_x;
   a.s_c = s_c;
   a.out = out;
@@ -366,7 +367,127 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   return out_i32 ? launch_gemm<true>(s, tx, tw, ts, ta, a, cs) : launch_gemm<false>(s, tx, tw, ts, ta, a, cs);
 }
 
+// ---------------------------------------- fused activation quantization
+// One launch does act-quant + GEMM when the automatic schedule is a split-K
+// cluster of 16-token tiles whose CTAs preload all of their K-blocks: every
+// CTA then holds its whole K-slice of the activations and the row maxima can
+// be combined over the cluster (see the FQ notes in lq_gemm_kernel.cuh).
+bool fused_eligible(const Schedule& s, int M) {
+  if (M < 1 || M > 16 || s.kind != kSchedTiles || s.bt != 16 || s.cs < 2) return false;
+  const int per_cta = (s.KB + s.cs - 1) / s.cs;  // the largest K-slice, in K-blocks
+  return per_cta <= lq::GemmCfg<16, 2>::kStages;
+}
+
+// The automatic choice: the four quantizing warps of a CTA take M/4 tokens
+// each, so the fused launch wins only while M is small (measured on B200 at
+// N = K = 4096: ahead up to M = 8, behind from M = 12).
+constexpr int kFusedAutoMaxM = 8;
+
+bool use_fused(const Schedule& s, int M, int path) {
+  if (path == LQ_LINEAR_TWO_LAUNCHES) return false;
+  if (!fused_eligible(s, M)) return false;
+  return path == LQ_LINEAR_FUSED || M <= kFusedAutoMaxM;
+}
+
+template <int CS>
+lq_status launch_fused_t(const Schedule& s, const CUtensorMap& tw, const CUtensorMap& ts, const CUtensorMap& ta,
+                         const lq::GemmArgs& a, cudaStream_t st) {
+  using C = lq::GemmCfg<16, CS>;
+  auto kern = lq::w4a8_gemm_kernel<16, CS, false, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  // no activation tensor map: the weight map stands in for it (never used)
+  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tw, tw, ts, ta, a);
+}
+
+size_t align16(size_t b) { return (b + 15) / 16 * 16; }
+
 }  // namespace
+
+extern "C" {
+
+size_t lq_w4a8_linear_workspace_size_ex(int M, int N, int K, int path) {
+  if (check_gemm_shape(M, N, K, LQ_GROUP) != LQ_OK || M == 0) return 0;
+  if (path < LQ_LINEAR_AUTO || path > LQ_LINEAR_FUSED) return 0;
+  DeviceInfo* dev = nullptr;
+  int sms = 148;
+  if (current_device(&dev) == LQ_OK) sms = dev->sms;
+  const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, sms);
+  if (use_fused(s, M, path)) return 0;
+  return align16((size_t)M * K) + align16((size_t)M * 4) + s.ws_bytes;
+}
+
+size_t lq_w4a8_linear_workspace_size(int M, int N, int K) {
+  return lq_w4a8_linear_workspace_size_ex(M, N, K, LQ_LINEAR_AUTO);
+}
+
+lq_status lq_w4a8_linear(const void* X_bf16, const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8,
+                         const float* s_c, void* out_bf16, int M, int N, int K, int group, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return lq_w4a8_linear_ex(X_bf16, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes,
+                           LQ_LINEAR_AUTO, stream);
+}
+
+lq_status lq_w4a8_linear_ex(const void* X_bf16, const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8,
+                            const float* s_c, void* out_bf16, int M, int N, int K, int group, void* workspace,
+                            size_t workspace_bytes, int path, void* stream) {
+  lq_status st = check_gemm_shape(M, N, K, group);
+  if (st != LQ_OK) return st;
+  if (path < LQ_LINEAR_AUTO || path > LQ_LINEAR_FUSED) return LQ_ERR_INVALID_ARG;
+  if (M == 0) return LQ_OK;
+  if (!X_bf16 || !qw || !s_u8 || !a_u8 || !s_c || !out_bf16) return LQ_ERR_INVALID_ARG;
+  if (!aligned(X_bf16, 16) || !aligned(qw, 16) || !aligned(s_u8, 16) || !aligned(a_u8, 16) ||
+      !aligned(out_bf16, 16) || !aligned(s_c, 4))
+    return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, dev->sms);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (path == LQ_LINEAR_FUSED && !fused_eligible(s, M)) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (!use_fused(s, M, path)) {
+    // two launches: activations into the workspace, then the GEMM
+    const size_t xq_bytes = align16((size_t)M * K), sx_bytes = align16((size_t)M * 4);
+    if (!workspace || workspace_bytes < xq_bytes + sx_bytes + s.ws_bytes) return LQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return LQ_ERR_MISALIGNED;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    int8_t* x_q = reinterpret_cast<int8_t*>(w);
+    float* s_x = reinterpret_cast<float*>(w + xq_bytes);
+    st = lq_quantize_act(X_bf16, M, K, x_q, s_x, stream);
+    if (st != LQ_OK) return st;
+    return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, w + xq_bytes + sx_bytes,
+                     workspace_bytes - xq_bytes - sx_bytes, 0, 0, 0, 0, false, stream);
+  }
+  CUtensorMap tw, ts, ta;
+  if (!make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, lq::kBlockK / 2, lq::kBlockN,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_u8(&ts, s_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, 2u,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_u8(&ta, a_u8, (uint64_t)N, (uint64_t)K / LQ_GROUP, (uint64_t)N, lq::kBlockN, 2u,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return LQ_ERR_CUDA;
+  lq::GemmArgs a;
+  a.x_bf16 = static_cast<const uint16_t*>(X_bf16);
+  a.s_x = nullptr;
+  a.s_c = s_c;
+  a.out = out_bf16;
+  a.ws = nullptr;
+  a.ticket = nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = s.tiles_m;
+  a.KB = s.KB;
+  a.U = s.U;
+  switch (s.cs) {
+    case 2: return launch_fused_t<2>(s, tw, ts, ta, a, cs);
+    case 4: return launch_fused_t<4>(s, tw, ts, ta, a, cs);
+    case 8: return launch_fused_t<8>(s, tw, ts, ta, a, cs);
+  }
+  return LQ_ERR_INVALID_ARG;
+}
+
+}  // extern "C"
 
 extern "C" {
 

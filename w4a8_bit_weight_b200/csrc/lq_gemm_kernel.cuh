@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 
 #include "lq_device.cuh"
+#include "lq_quant_kernels.cuh"
 
 namespace lq {
 
@@ -82,7 +83,9 @@ struct GemmCfg {
   static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * kOwned * kPieceBytes : 0;  // received pieces
   static constexpr int kXRing = kStages * kXBytes;
   static constexpr int kWRing = kStages * kWStage;
-  static constexpr int kBarBytes = 512;
+  // mbarriers and flags in the first 512 bytes; with fused activation
+  // quantization, the cluster's partial row maxima [CS][16] and s_x [16] after
+  static constexpr int kBarBytes = 1152;
   static constexpr int kUsed = kXRing + kWRing + kRedBytes + kBarBytes + 1024;  // + alignment slack
   // Shared memory also bounds how many CTAs share an SM: a 512-column CTA
   // takes at least 120 KB (one per SM), a 256-column CTA at least 80 KB (at
@@ -91,10 +94,12 @@ struct GemmCfg {
   static_assert(kAccCols + kSlots * 32 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kXBytes % 1024 == 0 && (kXRing + kWRing + kRedBytes) % 8 == 0, "alignment");
-  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 6 * 8 + 16 <= kBarBytes, "barrier area");
+  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 7 * 8 + 16 <= 512, "barrier area");
+  static_assert(512 + 8 * 16 * 4 + 16 * 4 <= kBarBytes, "fused-quantization area");
 };
 
 struct GemmArgs {
+  const uint16_t* x_bf16;  // fused activation quantization only: X [M, K] bf16
   const float* s_x;
   const float* s_c;
   void* out;             // bf16 [M, N] or int32 [M, N]
@@ -146,6 +151,20 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volat
   const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase, abort_flag));
   phase ^= 1u;
   return ok;
+}
+
+// Four bf16 (two words, in order) -> four INT8 codes, one word: the same codes as
+// quant_pair_i8 (rint(x * inv), then into [-127, 127]: the floor is applied
+// before the saturating pack, which supplies the ceiling).
+__device__ __forceinline__ uint32_t quant_quad_i8(uint32_t w01, uint32_t w23, float inv) {
+  const int i0 = max(-127, __float2int_rn(__fmul_rn(__uint_as_float(w01 << 16), inv)));
+  const int i1 = max(-127, __float2int_rn(__fmul_rn(__uint_as_float(w01 & 0xFFFF0000u), inv)));
+  const int i2 = max(-127, __float2int_rn(__fmul_rn(__uint_as_float(w23 << 16), inv)));
+  const int i3 = max(-127, __float2int_rn(__fmul_rn(__uint_as_float(w23 & 0xFFFF0000u), inv)));
+  uint32_t hi, r;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(i3), "r"(i2));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(i1), "r"(i0), "r"(hi));
+  return r;
 }
 
 // Writes TC consecutive tokens [m_first, m_first + TC) of this thread's output
@@ -212,12 +231,19 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&v)[32]
 
 // CTAs that keep to 256 TMEM columns are meant to share an SM with a CTA of
 // the next launch (programmatic dependent launch): registers are capped for two.
-template <int BT, int CS, bool OUT_I32>
+//
+// FQ (fused activation quantization, 16-token tiles in a split-K cluster whose
+// K-blocks all fit the preloaded stages): the activations arrive as bf16 and
+// the expansion warps quantize them (per-token symmetric INT8, the same
+// arithmetic as quantize_act_kernel) straight into the swizzled activation
+// tiles; the row maxima are combined over the cluster through DSMEM.
+template <int BT, int CS, bool OUT_I32, bool FQ = false>
 __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 256 ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
                      const GemmArgs p) {
   using C = GemmCfg<BT, CS>;
+  static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
   constexpr int S = C::kStages;
   constexpr int A = C::kSlots;
   constexpr int CH = BT < 32 ? BT : 32;  // accumulator columns per TMEM load
@@ -236,9 +262,12 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   uint64_t* grp = drain + 1;
   uint64_t* redbar = grp + 1;
   uint64_t* xfirst = redbar + 1;  // the activation tiles of the first min(S, total) K-blocks, all at once
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xfirst + 1);
+  uint64_t* amaxbar = xfirst + 1;  // FQ: the other CTAs' partial row maxima have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(amaxbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  float* amx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(wfull) + 512);  // FQ: [CS][16]
+  float* sxs = amx + 8 * 16;                                                       // FQ: s_x [16]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -260,7 +289,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     // every CTA of a split-K cluster expects its piece from each of the others
     mbar_init(redbar, 1);
     if (CS >= 2) mbar_arrive_expect_tx(redbar, (uint32_t)C::kRedBytes);
-    mbar_init(xfirst, 1);
+    mbar_init(xfirst, FQ ? 4 : 1);  // FQ: the four quantizing warps
+    mbar_init(amaxbar, 1);
+    if (FQ) mbar_arrive_expect_tx(amaxbar, (uint32_t)(CS - 1) * 16 * 4);
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -330,7 +361,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       }
     }
     griddep_wait();
-    if (leader && P > 0) {
+    if (leader && P > 0 && !FQ) {
       // one barrier for all of them: the MMA warp waits once
       mbar_arrive_expect_tx(xfirst, (uint32_t)P * C::kTxX);
       UnitCursor cx = first;
@@ -367,7 +398,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     if (leader && *abort_flag) {
       // never leave a bulk copy in flight into shared memory that is about to be released
       const unsigned long long t0w = globaltimer();
-      if (P > 0)
+      if (P > 0 && !FQ)
         while (!mbar_try_wait(smem_u32(xfirst), 0) && globaltimer() - t0w < 100000000ull) {
         }
       for (int s = 0; s < S; ++s) {
@@ -466,12 +497,129 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     bool red_done = !(CS >= 2 && (CS >= 4 ? sub == (int)crank / C::kSlices : sub / C::kOwned == (int)crank));
     int stage = 0, slot = 0;
     uint32_t sphase = 0, aphase = 0;
+
+    // ------------------------------------------ fused activation quantization
+    // (FQ) Quantizes this CTA's K-slice of the tile's activations into the
+    // activation tiles.  Warp e = warp - 2 takes tokens e, e+4, e+8, e+12 (a
+    // small batch spreads over all four warps; the cluster's partial maxima
+    // are kept per warp, amx[src][4e + i] for token e + 4i), lane l the
+    // 32 consecutive K of chunk l (a 128-K block is four chunks; the slice has
+    // at most S blocks, so one chunk per lane at most).  Runs once the weight
+    // blocks that have a slot of their own are expanded: the next block
+    // waits for an MMA, and the MMAs wait for this.
+    const int total_e = (int)(u_end - u_begin);
+    bool x_done = !FQ;
+    auto fused_quantize = [&]() -> bool {
+      x_done = true;
+      griddep_wait();  // X may be the output of the preceding kernel
+      waited_dep = true;
+      cluster_wait();  // the other CTAs' barriers exist before any remote store
+      cl_waited = true;
+      const int e = warp - 2;
+      const int nchunk = total_e * (kBlockK / 32);
+      const int k0 = (int)(u_begin - (u_begin / KB) * KB) * kBlockK + lane * 32;  // this lane's first K
+      const bool has = lane < nchunk;
+      // the four tokens are independent: all loads first, then the reductions
+      // and divisions side by side, so that no chain waits on another
+      uint4 xv[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int m = e + 4 * i;
+        const bool ld = has && m < p.M;
+        const uint4* src = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)(ld ? m : 0) * p.K + (ld ? k0 : 0));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) xv[i][c] = ld ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float pm[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        // max |x| on bf16 pairs: bf16 -> fp32 is exact and monotone, so the
+        // maximum is the same as over the fp32 values
+        __nv_bfloat162 m2 = __floats2bfloat162_rn(0.0f, 0.0f);
+        if (e + 4 * i < p.M) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t w4[4] = {xv[i][c].x, xv[i][c].y, xv[i][c].z, xv[i][c].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w4[j])));
+          }
+        }
+        const uint32_t mb = *reinterpret_cast<const uint32_t*>(&m2);
+        pm[i] = fmaxf(bf16_bits_to_f32(mb & 0xFFFFu), bf16_bits_to_f32(mb >> 16));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pm[i] = fmaxf(pm[i], __shfl_xor_sync(0xffffffffu, pm[i], o));
+      // pm[i]: this CTA's maximum of |X[4e + i, slice]|.  Partial maxima to the
+      // other CTAs of the cluster (16 bytes each, counted on their barrier)
+      // and to this CTA's own row.
+      if (lane == 0) {
+        *reinterpret_cast<float4*>(amx + crank * 16 + 4 * e) = make_float4(pm[0], pm[1], pm[2], pm[3]);
+#pragma unroll
+        for (int o = 0; o < CS; ++o)
+          if (o != (int)crank)
+            st_async_v4(mapa_shared(smem_u32(amx + crank * 16 + 4 * e), (uint32_t)o), __float_as_uint(pm[0]),
+                        __float_as_uint(pm[1]), __float_as_uint(pm[2]), __float_as_uint(pm[3]),
+                        mapa_shared(smem_u32(amaxbar), (uint32_t)o));
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(amaxbar, 0, abort_flag))) return false;
+      // lane i < 4 finishes token 4e + i (row maximum over the cluster, the two
+      // IEEE divisions) and hands 127/amax to the warp
+      float inv_l = 0.0f;
+      if (lane < 4) {
+        const int m = e + 4 * lane;
+        float a = lane == 0 ? pm[0] : lane == 1 ? pm[1] : lane == 2 ? pm[2] : pm[3];
+#pragma unroll
+        for (int o = 0; o < CS; ++o)
+          if (o != (int)crank) a = fmaxf(a, amx[o * 16 + 4 * e + lane]);
+        const bool zero = (a == 0.0f);
+        inv_l = zero ? 0.0f : __fdiv_rn(127.0f, a);
+        sxs[m] = zero ? 1.0f : __fdiv_rn(a, 127.0f);
+      }
+      float inv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) inv[i] = __shfl_sync(0xffffffffu, inv_l, i);
+      if (has) {
+        // lane l: 32 codes of each token = two 16-byte chunks of its row in
+        // block l / 4 (128-byte swizzle)
+        uint8_t* blk = xring + (size_t)(lane >> 2) * C::kXBytes;
+        const int ch = (lane & 3) * 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = e + 4 * i;
+          uint32_t q[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // rows past the batch stay zero
+          if (m < p.M) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              q[2 * c] = quant_quad_i8(xv[i][c].x, xv[i][c].y, inv[i]);
+              q[2 * c + 1] = quant_quad_i8(xv[i][c].z, xv[i][c].w, inv[i]);
+            }
+          }
+          uint8_t* row = blk + m * 128;
+          *reinterpret_cast<uint4*>(row + ((ch ^ (m & 7)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+          *reinterpret_cast<uint4*>(row + (((ch + 1) ^ (m & 7)) << 4)) = make_uint4(q[4], q[5], q[6], q[7]);
+        }
+      }
+      // the tensor core reads these tiles through the async proxy
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xfirst);
+      return true;
+    };
+    int it_e = 0;
+    const int x_at = min(A, total_e);  // the first block that waits for an MMA (or the end)
+
     for (long long u = u_begin; u < u_end;) {
       const int t = (int)(u / KB);
       const int kb0 = (int)(u % KB);
       const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
       const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb, ++it_e) {
+        if constexpr (FQ) {
+          if (it_e == x_at && !fused_quantize()) goto epi_done;
+        }
         // warp-uniform decision: every lane waits, all continue only if all saw the phase
         if (!__all_sync(0xffffffffu, mbar_wait(&wfull[stage], sphase, abort_flag) &&
                                          mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag)))
@@ -509,6 +657,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
         }
       }
 
+      if constexpr (FQ) {
+        if (!x_done && !fused_quantize()) goto epi_done;
+      }
       // ------------------------------------------------------- epilogue
       if (!waited_dep) {
         griddep_wait();  // scales and the output may belong to the preceding kernel
@@ -523,7 +674,14 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       // the first token this warp writes: split-K clusters write only their own piece
       constexpr int SXC = CS >= 2 ? (C::kPieceT < 32 ? C::kPieceT : 32) : CH;
       const int sx0 = m0 + (CS >= 4 ? (int)(crank % C::kSlices) * C::kPieceT : 0);
-      float sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
+      float sx_next = 0.0f;
+      if constexpr (FQ) {
+        // s_x from the quantizing warps (all four have arrived on xfirst)
+        if (!__all_sync(0xffffffffu, mbar_wait(xfirst, 0, abort_flag))) goto epi_done;
+        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? sxs[sx0 - m0 + lane] : 0.0f;
+      } else {
+        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
       acc_phase ^= 1u;
       tc_fence_after();
@@ -535,8 +693,10 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           constexpr int TC = T < 32 ? T : 32;  // TMEM columns per load
           const int q = sub;                   // this warp's row quarter
           // the other CTAs' barriers are initialized once the whole cluster has arrived
-          cluster_wait();
-          cl_waited = true;
+          if (!cl_waited) {
+            cluster_wait();
+            cl_waited = true;
+          }
           // 1. pieces owned by other CTAs: TMEM -> this warp's staging rows
           //    [token][lane] (in the free activation ring) -> one bulk copy each
           uint32_t* stg = reinterpret_cast<uint32_t*>(xring) + (size_t)q * BT * 32;
@@ -586,7 +746,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
               const float sx_cur = sx_next;
               if (c + 1 < T / TC) {
                 const int mn = m0 + h * T + (c + 1) * TC + lane;
-                sx_next = (!OUT_I32 && lane < TC && mn < p.M) ? __ldg(p.s_x + mn) : 0.0f;
+                sx_next = (!OUT_I32 && lane < TC && mn < p.M) ? (FQ ? sxs[mn - m0] : __ldg(p.s_x + mn)) : 0.0f;
               }
               uint32_t v[32];
               const uint32_t col = (uint32_t)(h * T + c * TC);
