@@ -128,7 +128,11 @@ LQ_API lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, 
  *   before that kernel has finished, so those buffers must not be written by
  *   a kernel that itself triggers early launch (this library's weight
  *   quantizer does not); x_q, s_x, s_c and out are touched only after it has
- *   completed.
+ *   completed.  Each GEMM and lq_quantize_act in turn lets the next kernel in
+ *   the stream launch as soon as its own CTAs have started: a kernel launched
+ *   after it with programmatic stream serialization must wait for it
+ *   (griddepcontrol.wait) before reading its output; other kernels are
+ *   ordered as usual.
  */
 LQ_API size_t lq_w4a8_gemm_workspace_size(int M, int N, int K);
 LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw,
