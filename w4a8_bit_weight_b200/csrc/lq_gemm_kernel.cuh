@@ -455,14 +455,35 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           // the whole run back to back, one thread, no warp synchronization
           tc_fence_after();
           int stage = it % S, slot = it % A;
-          for (int r = 0; r < run; ++r) {
+          // K-blocks whose stage (and slot) a later block reuses need release
+          // commits, those whose slot only is reused need one, the rest none:
+          // three loops, so that the last is a plain run of MMAs (measurably
+          // faster to issue than one loop with the conditions inside)
+          const int r_both = min(run, max(0, total - S - it));
+          const int r_slot = min(run, max(0, total - A - it));
+          auto issue = [&](int r) {
             const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
             const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
 #pragma unroll
             for (int j = 0; j < kBlockK / 32; ++j)
               mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb + r > kb0 || j > 0) ? 1u : 0u);
-            if (it + r + S < total) tc_commit(&empty[stage]);
-            if (it + r + A < total) tc_commit(&aempty[slot]);
+          };
+          int r = 0;
+          for (; r < r_both; ++r) {
+            issue(r);
+            tc_commit(&empty[stage]);
+            tc_commit(&aempty[slot]);
+            if (++stage == S) stage = 0;
+            if (++slot == A) slot = 0;
+          }
+          for (; r < r_slot; ++r) {
+            issue(r);
+            tc_commit(&aempty[slot]);
+            if (++stage == S) stage = 0;
+            if (++slot == A) slot = 0;
+          }
+          for (; r < run; ++r) {
+            issue(r);
             if (++stage == S) stage = 0;
             if (++slot == A) slot = 0;
           }
