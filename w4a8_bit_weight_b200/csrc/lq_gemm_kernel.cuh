@@ -513,9 +513,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     const int sw = (r >> 1) & 3;        // 64-byte swizzle of this row's 16-byte chunks
     uint32_t acc_phase = 0, grp_phase = 0;
     bool waited_dep = false;
-    // split-K: the warps that own a piece must see all of it arrive before the
-    // CTA may leave (the others' bulk copies write into this CTA)
-    bool red_done = !(CS >= 2 && (CS >= 4 ? sub == (int)crank / C::kSlices : sub / C::kOwned == (int)crank));
+    // split-K: every epilogue warp reads this CTA's piece, so each must see all
+    // of it arrive before the CTA may leave (the others' bulk copies write here)
+    bool red_done = (CS < 2);
     int stage = 0, slot = 0;
     uint32_t sphase = 0, aphase = 0;
 
@@ -718,32 +718,33 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
             cluster_wait();
             cl_waited = true;
           }
-          // 1. pieces owned by other CTAs: TMEM -> this warp's staging rows
-          //    [token][lane] (in the free activation ring) -> one bulk copy each
+          // 1. this warp's quarter of the partial sums: TMEM -> staging rows
+          //    [token][lane] in the free activation ring
           uint32_t* stg = reinterpret_cast<uint32_t*>(xring) + (size_t)q * BT * 32;
+#pragma unroll 1
+          for (int c = 0; c < BT / TC; ++c) {
+            uint32_t v[32];
+            const uint32_t col = (uint32_t)(c * TC);
+            if constexpr (TC == 8) {
+              uint32_t v8[8];
+              tmem_ld_32x32b_x8(t_lane + col, v8);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) v[i] = v8[i];
+            } else {
+              tmem_load_cols<TC>(t_lane + col, v);
+            }
+#pragma unroll
+            for (int i = 0; i < TC; ++i) stg[(col + i) * 32 + lane] = v[i];
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          // 2. the pieces other CTAs own: one bulk copy each, counted on the owner's barrier
           bool sent = false;
 #pragma unroll 1
           for (int h = 0; h < C::kSlices; ++h) {
             const int o = CS >= 4 ? q * C::kSlices + h : q / C::kOwned;
             if (o == (int)crank) continue;
-#pragma unroll 1
-            for (int c = 0; c < T / TC; ++c) {
-              uint32_t v[32];
-              const uint32_t col = (uint32_t)(h * T + c * TC);
-              if constexpr (TC == 8) {
-                uint32_t v8[8];
-                tmem_ld_32x32b_x8(t_lane + col, v8);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = v8[i];
-              } else {
-                tmem_load_cols<TC>(t_lane + col, v);
-              }
-#pragma unroll
-              for (int i = 0; i < TC; ++i) stg[(col + i) * 32 + lane] = v[i];
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
             if (lane == 0) {
               const int slot = (int)crank < o ? (int)crank : (int)crank - 1;
               const int pidx = CS >= 4 ? 0 : q % C::kOwned;
@@ -753,40 +754,42 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
             }
             sent = true;
           }
-          // 2. the piece this warp owns, if any: own partial + the others' pieces
-#pragma unroll 1
-          for (int h = 0; h < C::kSlices; ++h) {
-            const int o = CS >= 4 ? q * C::kSlices + h : q / C::kOwned;
-            if (o != (int)crank) continue;
-            // every lane observes the completed bytes itself (cluster-scope acquire)
-            if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
-            red_done = true;
-            const int pidx = CS >= 4 ? 0 : q % C::kOwned;
-#pragma unroll 1
-            for (int c = 0; c < T / TC; ++c) {
-              const float sx_cur = sx_next;
-              if (c + 1 < T / TC) {
-                const int mn = m0 + h * T + (c + 1) * TC + lane;
-                sx_next = (!OUT_I32 && lane < TC && mn < p.M) ? (FQ ? sxs[mn - m0] : __ldg(p.s_x + mn)) : 0.0f;
-              }
-              uint32_t v[32];
-              const uint32_t col = (uint32_t)(h * T + c * TC);
-              if constexpr (TC == 8) {
-                uint32_t v8[8];
-                tmem_ld_32x32b_x8(t_lane + col, v8);
-                tmem_ld_wait();
+          // 3. this CTA's own piece, shared by all four warps: the owning
+          //    warp's staged partial (visible after the group barrier) plus
+          //    the others' pieces (visible after their bytes have landed)
+          if (!group_sync(grp, grp_phase, abort_flag)) goto epi_done;
+          // every lane observes the completed bytes itself (cluster-scope acquire)
+          if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
+          red_done = true;
+          {
+            constexpr int kWarpsPerPiece = 4 / C::kOwned;     // CS = 2: two quarters, two warps each
+            constexpr int kTok = T / kWarpsPerPiece;          // tokens per thread
+            const int e = warp - 2;
+            const int pidx = CS >= 4 ? 0 : e % C::kOwned;
+            const int qq = CS >= 4 ? (int)crank / C::kSlices : (int)crank * C::kOwned + pidx;  // owned quarter
+            const int hh = CS >= 4 ? (int)crank % C::kSlices : 0;                              // owned token slice
+            const int t0 = CS >= 4 ? e : e / C::kOwned;
+            const int nn = tile_n * kBlockN + qq * 32 + lane;
+            const bool nn_ok = nn < p.N;
+            const float scn = (!OUT_I32 && nn_ok) ? __ldg(p.s_c + nn) : 0.0f;
+            const uint32_t* own = reinterpret_cast<const uint32_t*>(xring) + (size_t)qq * BT * 32 + (size_t)hh * T * 32;
+#pragma unroll 4
+            for (int i = 0; i < kTok; ++i) {
+              const int t = t0 + i * kWarpsPerPiece;  // token within the piece
+              const int m = m0 + hh * T + t;
+              uint32_t acc = own[t * 32 + lane];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = v8[i];
-              } else {
-                tmem_load_cols<TC>(t_lane + col, v);
+              for (int sidx = 0; sidx < CS - 1; ++sidx)
+                acc += (uint32_t)red[((size_t)sidx * C::kOwned + pidx) * T * 32 + t * 32 + lane];
+              if (m < p.M && nn_ok) {
+                if constexpr (OUT_I32) {
+                  reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + nn] = (int32_t)acc;
+                } else {
+                  const float sxm = FQ ? sxs[m - m0] : __ldg(p.s_x + m);
+                  const float y = __fmul_rn(__int2float_rn((int32_t)acc), __fmul_rn(sxm, scn));
+                  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + nn] = __float2bfloat16_rn(y);
+                }
               }
-#pragma unroll
-              for (int sidx = 0; sidx < CS - 1; ++sidx) {
-                const int32_t* rp = red + ((size_t)sidx * C::kOwned + pidx) * T * 32 + (size_t)c * TC * 32 + lane;
-#pragma unroll
-                for (int i = 0; i < TC; ++i) v[i] += (uint32_t)rp[i * 32];
-              }
-              store_chunk<OUT_I32, TC>(p, m0 + h * T + c * TC, n, n_ok, v, sx_cur, sc);
             }
           }
           tc_fence_before();
