@@ -94,7 +94,12 @@ struct GemmCfg {
   static_assert(kAccCols + kSlots * 32 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kXBytes % 1024 == 0 && (kXRing + kWRing + kRedBytes) % 8 == 0, "alignment");
-  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 7 * 8 + 16 <= 512, "barrier area");
+  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 8 * 8 + 16 <= 512, "barrier area");
+  // One K-block more than TMEM slots and no refills (a 16- or 32-token decode
+  // CTA holding its whole K-slice): the extra block is expanded into the
+  // shared memory of weight stages 0-1 (free by then) and multiplied with A
+  // from shared memory, instead of waiting for slot 0 to be released.
+  static_assert(kSlots < 2 || 128 * kBlockK <= 2 * kWStage, "overflow block fits two weight stages");
   static_assert(512 + 8 * 16 * 4 + 16 * 4 <= kBarBytes, "fused-quantization area");
 };
 
@@ -263,7 +268,8 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   uint64_t* redbar = grp + 1;
   uint64_t* xfirst = redbar + 1;  // the activation tiles of the first min(S, total) K-blocks, all at once
   uint64_t* amaxbar = xfirst + 1;  // FQ: the other CTAs' partial row maxima have landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(amaxbar + 1);
+  uint64_t* ovfull = amaxbar + 1;  // the overflow K-block is expanded in shared memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ovfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float* amx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(wfull) + 512);  // FQ: [CS][16]
@@ -291,6 +297,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     if (CS >= 2) mbar_arrive_expect_tx(redbar, (uint32_t)C::kRedBytes);
     mbar_init(xfirst, FQ ? 4 : 1);  // FQ: the four quantizing warps
     mbar_init(amaxbar, 1);
+    mbar_init(ovfull, 4);
     if (FQ) mbar_arrive_expect_tx(amaxbar, (uint32_t)(CS - 1) * 16 * 4);
     *abort_flag = 0;
     *last_flag = 0;
@@ -331,6 +338,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     u_begin = (long long)blockIdx.x * U / G;
     u_end = ((long long)blockIdx.x + 1) * U / G;
   }
+
+  // the overflow K-block (see GemmCfg): one tile, exactly one block more than slots, no refills
+  const bool ovf = CS >= 1 && A >= 2 && (int)(u_end - u_begin) == A + 1 && A + 1 <= S;
 
   // Producer and MMA warps run their loops with all 32 lanes (one lane issues),
   // so every warp stays converged up to the CTA barrier at teardown.
@@ -439,13 +449,17 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
             ok = mbar_wait(&xfull[stage], (uint32_t)(it / S - 1) & 1u, abort_flag);
           }
           if (ok && it >= ready) {
-            ok = mbar_wait(&afull[slot], (uint32_t)(it / A) & 1u, abort_flag);
+            ok = (ovf && it == A) ? mbar_wait(ovfull, 0, abort_flag)
+                                  : mbar_wait(&afull[slot], (uint32_t)(it / A) & 1u, abort_flag);
             ready = it + 1;
             // inside the window of preloaded stages the expansion usually runs
             // ahead (it works while this kernel waits for its inputs): one look
             // at the furthest block there may cover all the blocks before it
             const int hi = min(it + A - 1, P - 1);
-            if (ok && hi > it && mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u)) ready = hi + 1;
+            if (ok && hi > it && (!ovf || hi < A) &&
+                mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u))
+              ready = hi + 1;
+            if (ok && ovf && ready == A && mbar_try_wait(smem_u32(ovfull), 0)) ready = A + 1;
           }
           run = min(min(ready, it < P ? P : it + 1) - it, kb1 - kb);
         }
@@ -459,8 +473,11 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           // commits, those whose slot only is reused need one, the rest none:
           // three loops, so that the last is a plain run of MMAs (measurably
           // faster to issue than one loop with the conditions inside)
-          const int r_both = min(run, max(0, total - S - it));
-          const int r_slot = min(run, max(0, total - A - it));
+          // the overflow block, if this run reaches it, goes last and separately
+          const bool run_ovf = ovf && it + run == A + 1;
+          const int run_ts = run - (run_ovf ? 1 : 0);
+          const int r_both = min(run_ts, max(0, total - S - it));
+          const int r_slot = min(run_ts, max(0, total - A - it));
           auto issue = [&](int r) {
             const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
             const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
@@ -482,10 +499,17 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
             if (++stage == S) stage = 0;
             if (++slot == A) slot = 0;
           }
-          for (; r < run; ++r) {
+          for (; r < run_ts; ++r) {
             issue(r);
             if (++stage == S) stage = 0;
             if (++slot == A) slot = 0;
+          }
+          if (run_ovf) {
+            const uint64_t adesc = smem_desc_k_sw128(smem_u32(wring));
+            const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
+#pragma unroll
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_i8_ss(tmem_base, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, 1u);
           }
         }
         it += run;
@@ -630,7 +654,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       return true;
     };
     int it_e = 0;
-    const int x_at = min(A, total_e);  // the first block that waits for an MMA (or the end)
+    // the first block that waits for an MMA (or the end; with the overflow
+    // block in shared memory no block does)
+    const int x_at = ovf ? total_e : min(A, total_e);
 
     for (long long u = u_begin; u < u_end;) {
       const int t = (int)(u / KB);
@@ -641,9 +667,13 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
         if constexpr (FQ) {
           if (it_e == x_at && !fused_quantize()) goto epi_done;
         }
+        // the overflow block goes to shared memory: it needs weight stages 0-1,
+        // which every warp has finished reading once block 1 is expanded
+        const bool to_smem = ovf && it_e == A;
         // warp-uniform decision: every lane waits, all continue only if all saw the phase
         if (!__all_sync(0xffffffffu, mbar_wait(&wfull[stage], sphase, abort_flag) &&
-                                         mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag)))
+                                         (to_smem ? mbar_wait(&afull[1], 0, abort_flag)
+                                                  : mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag))))
           goto epi_done;
         tc_fence_after();
         const uint8_t* wb = wring + stage * C::kWStage;
@@ -663,11 +693,22 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
           lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
         }
-        tmem_st_32x32b_x32(t_lane + C::kAccCols + slot * 32, v);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[slot]);
+        if (to_smem) {
+          // row r of a 128-byte-swizzled K-major tile (the MMA's A descriptor)
+          uint8_t* orow = wring + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(orow + ((c ^ (r & 7)) << 4)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          fence_proxy_async_smem();  // read by the tensor core through the async proxy
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ovfull);
+        } else {
+          tmem_st_32x32b_x32(t_lane + C::kAccCols + slot * 32, v);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[slot]);
+        }
         if (++stage == S) {
           stage = 0;
           sphase ^= 1u;
