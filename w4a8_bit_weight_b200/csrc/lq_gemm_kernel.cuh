@@ -744,6 +744,32 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       } else {
         sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
       }
+      // split-K clusters: the scales of the piece this thread will write (the
+      // reduce-scatter's owner phase), also loaded before the accumulator wait
+      constexpr int kWarpsPerPiece = 4 / C::kOwned;         // CS = 2: two quarters, two warps each
+      constexpr int kTok = C::kPieceT / kWarpsPerPiece;     // tokens per thread in the owner phase
+      constexpr int kTokPre = (CS >= 2 && kTok <= 8) ? kTok : 1;
+      const int oe = warp - 2;
+      const int opidx = CS >= 4 ? 0 : oe % C::kOwned;
+      const int oqq = CS >= 4 ? (int)crank / C::kSlices : (int)crank * C::kOwned + opidx;  // owned quarter
+      const int ohh = CS >= 4 ? (int)crank % C::kSlices : 0;                               // owned token slice
+      const int ot0 = CS >= 4 ? oe : oe / C::kOwned;
+      const int onn = tile_n * kBlockN + oqq * 32 + lane;
+      const bool onn_ok = onn < p.N;
+      float oscn = 0.0f;
+      float osx[kTokPre];
+#pragma unroll
+      for (int i = 0; i < kTokPre; ++i) osx[i] = 0.0f;
+      if constexpr (CS >= 2 && !OUT_I32) {
+        oscn = onn_ok ? __ldg(p.s_c + onn) : 0.0f;
+        if constexpr (kTok <= 8) {
+#pragma unroll
+          for (int i = 0; i < kTok; ++i) {
+            const int m = m0 + ohh * C::kPieceT + ot0 + i * kWarpsPerPiece;
+            osx[i] = (m < p.M) ? (FQ ? sxs[m - m0] : __ldg(p.s_x + m)) : 0.0f;
+          }
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
       acc_phase ^= 1u;
       tc_fence_after();
@@ -803,32 +829,24 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
           red_done = true;
           {
-            constexpr int kWarpsPerPiece = 4 / C::kOwned;     // CS = 2: two quarters, two warps each
-            constexpr int kTok = T / kWarpsPerPiece;          // tokens per thread
-            const int e = warp - 2;
-            const int pidx = CS >= 4 ? 0 : e % C::kOwned;
-            const int qq = CS >= 4 ? (int)crank / C::kSlices : (int)crank * C::kOwned + pidx;  // owned quarter
-            const int hh = CS >= 4 ? (int)crank % C::kSlices : 0;                              // owned token slice
-            const int t0 = CS >= 4 ? e : e / C::kOwned;
-            const int nn = tile_n * kBlockN + qq * 32 + lane;
-            const bool nn_ok = nn < p.N;
-            const float scn = (!OUT_I32 && nn_ok) ? __ldg(p.s_c + nn) : 0.0f;
-            const uint32_t* own = reinterpret_cast<const uint32_t*>(xring) + (size_t)qq * BT * 32 + (size_t)hh * T * 32;
+            const uint32_t* own = reinterpret_cast<const uint32_t*>(xring) + (size_t)oqq * BT * 32 + (size_t)ohh * T * 32;
 #pragma unroll 4
             for (int i = 0; i < kTok; ++i) {
-              const int t = t0 + i * kWarpsPerPiece;  // token within the piece
-              const int m = m0 + hh * T + t;
+              const int t = ot0 + i * kWarpsPerPiece;  // token within the piece
+              const int m = m0 + ohh * T + t;
               uint32_t acc = own[t * 32 + lane];
 #pragma unroll
               for (int sidx = 0; sidx < CS - 1; ++sidx)
-                acc += (uint32_t)red[((size_t)sidx * C::kOwned + pidx) * T * 32 + t * 32 + lane];
-              if (m < p.M && nn_ok) {
+                acc += (uint32_t)red[((size_t)sidx * C::kOwned + opidx) * T * 32 + t * 32 + lane];
+              if (m < p.M && onn_ok) {
                 if constexpr (OUT_I32) {
-                  reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + nn] = (int32_t)acc;
+                  reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + onn] = (int32_t)acc;
                 } else {
-                  const float sxm = FQ ? sxs[m - m0] : __ldg(p.s_x + m);
-                  const float y = __fmul_rn(__int2float_rn((int32_t)acc), __fmul_rn(sxm, scn));
-                  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + nn] = __float2bfloat16_rn(y);
+                  float sxm;
+                  if constexpr (kTok <= 8) sxm = osx[i];
+                  else sxm = FQ ? sxs[m - m0] : __ldg(p.s_x + m);
+                  const float y = __fmul_rn(__int2float_rn((int32_t)acc), __fmul_rn(sxm, oscn));
+                  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + onn] = __float2bfloat16_rn(y);
                 }
               }
             }
