@@ -138,6 +138,18 @@ bool valid_schedule(int M, int block_t, int schedule, int split_k, int grid) {
   return false;
 }
 
+// shared-memory stages of the tile kernel for a token-tile size (one per
+// preloaded K-block of 128)
+int stages_of(int bt) {
+  switch (bt) {
+    case 16: return lq::GemmCfg<16, 1>::kStages;
+    case 32: return lq::GemmCfg<32, 1>::kStages;
+    case 64: return lq::GemmCfg<64, 1>::kStages;
+    case 128: return lq::GemmCfg<128, 2>::kStages;
+    default: return lq::GemmCfg<256, 1>::kStages;
+  }
+}
+
 Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms) {
   Schedule s;
   int kind = schedule;
@@ -201,13 +213,24 @@ Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split
   }
   int cs = split_k;
   if (cs <= 0) {
-    // one wave: as many CTAs per tile as fit on the SMs, at least 4 K-blocks each
+    // one wave of one CTA per SM: as many CTAs per tile as fit, at least 4
+    // K-blocks each.  That leaves room beside every CTA for one of the next
+    // launch, which preloads its weights meanwhile.
     cs = 1;
     for (int c = max_split(s.bt); c >= 2; c /= 2)
       if (s.tiles * c <= sms && s.KB / c >= 4) {
         cs = c;
         break;
       }
+    // When a CTA's K-slice is longer than its preloaded stages, the ring
+    // streams the rest anyway and more CTAs stream faster: tiles of up to 64
+    // tokens fit two CTAs per SM (256 TMEM columns), so use that capacity.
+    if (s.KB / cs > stages_of(s.bt) && s.bt <= 64)
+      for (int c = max_split(s.bt); c > cs; c /= 2)
+        if (s.tiles * c <= 2LL * sms && s.KB / c >= 4) {
+          cs = c;
+          break;
+        }
   }
   if (cs > s.KB) cs = 1;
   s.cs = cs;
