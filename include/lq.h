@@ -157,8 +157,8 @@ LQ_API lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t
  *               computed by a thread-block cluster of split_k CTAs, each
  *               summing one slice of the K-blocks of 128; partial sums are
  *               reduced through distributed shared memory.  split_k is 1, 2,
- *               4 or 8 (8 only for block_t <= 32, 4 for block_t <= 64, 2 for
- *               block_t <= 128, 1 for 256); 0 = automatic.  grid must be 0.
+ *               4 or 8 (8 only for block_t <= 32, 4 for block_t <= 128, 1
+ *               for 256); 0 = automatic.  grid must be 0.
  *             LQ_SCHED_PERSISTENT: grid CTAs (0 = one per SM) loop over the
  *               tiles, overlapping each tile's epilogue with the next tile's
  *               main loop.  split_k must be 0.

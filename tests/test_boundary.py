@@ -54,6 +54,7 @@ def gemm(lib, M=16, N=256, K=512, group=64, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=
     (dict(sched=1, split=2, grid=4), 1),          # a cluster split has no grid
     (dict(sched=3, split=2, grid=4), 1),          # stream-K has no cluster split
     (dict(sched=1, bt=64, split=8), 1),           # split 8 only for tiles of <= 32 tokens
+    (dict(sched=1, bt=128, split=8), 1),
     (dict(sched=1, bt=256, split=2), 1),          # 256-token tiles are never split
     (dict(sched=2, bt=64), 1),                    # the persistent schedule uses 128-token tiles
     (dict(sched=4, bt=128), 1),                   # CTA pairs use 256-token tiles

@@ -119,6 +119,7 @@ SHAPES = [
     (32, 256, 1152, 32, T, 8, 0),         # 9 K-blocks over 8 CTAs: uneven slices
     (40, 384, 1024, 64, T, 4, 0),
     (100, 256, 640, 128, T, 2, 0),
+    (100, 384, 1152, 128, T, 4, 0),       # 128-token tiles, 4-CTA clusters: 9 K-blocks unevenly
     (128, 384, 256, 128, T, 0, 0),
     (300, 256, 512, 256, T, 0, 0),        # ragged M with 256-token tiles
     (128, 128, 128, 0, P, 0, 0),          # persistent: one tile

@@ -108,7 +108,7 @@ int auto_block_t(int M) {
 bool valid_block_t(int bt) { return bt == 16 || bt == 32 || bt == 64 || bt == 128 || bt == 256; }
 
 // largest cluster split instantiated for a tile width (shared-memory bound)
-int max_split(int bt) { return bt <= 32 ? 8 : bt == 64 ? 4 : bt == 128 ? 2 : 1; }
+int max_split(int bt) { return bt <= 32 ? 8 : bt <= 128 ? 4 : 1; }
 
 bool valid_split(int bt, int cs) { return (cs == 1 || cs == 2 || cs == 4 || cs == 8) && cs <= max_split(bt); }
 
@@ -300,7 +300,7 @@ lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const CUtenso
       if constexpr (BT <= 128) return launch_gemm_t<BT, 2, I32>(s, tx, tw, ts, ta, a, st);
       break;
     case 4:
-      if constexpr (BT <= 64) return launch_gemm_t<BT, 4, I32>(s, tx, tw, ts, ta, a, st);
+      if constexpr (BT <= 128) return launch_gemm_t<BT, 4, I32>(s, tx, tw, ts, ta, a, st);
       break;
     case 8:
       if constexpr (BT <= 32) return launch_gemm_t<BT, 8, I32>(s, tx, tw, ts, ta, a, st);

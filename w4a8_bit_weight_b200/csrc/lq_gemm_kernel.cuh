@@ -84,7 +84,8 @@ struct GemmCfg {
   static constexpr int kXRing = kStages * kXBytes;
   static constexpr int kWRing = kStages * kWStage;
   // mbarriers and flags in the first 512 bytes; with fused activation
-  // quantization, the cluster's partial row maxima [CS][16] and s_x [16] after
+  // quantization, the cluster's partial row maxima [CS][16] and s_x [16]
+  // after; the expansion warps' progress counters [4] at byte 1088
   static constexpr int kBarBytes = 1152;
   static constexpr int kUsed = kXRing + kWRing + kRedBytes + kBarBytes + 1024;  // + alignment slack
   // Shared memory also bounds how many CTAs share an SM: a 512-column CTA
@@ -100,7 +101,7 @@ struct GemmCfg {
   // shared memory of weight stages 0-1 (free by then) and multiplied with A
   // from shared memory, instead of waiting for slot 0 to be released.
   static_assert(kSlots < 2 || 128 * kBlockK <= 2 * kWStage, "overflow block fits two weight stages");
-  static_assert(512 + 8 * 16 * 4 + 16 * 4 <= kBarBytes, "fused-quantization area");
+  static_assert(512 + 8 * 16 * 4 + 16 * 4 <= 1088 && 1088 + 4 * 4 <= kBarBytes, "fused-quantization and progress area");
 };
 
 struct GemmArgs {
@@ -251,6 +252,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
   constexpr int S = C::kStages;
   constexpr int A = C::kSlots;
+  // with as many TMEM slots as stages, block `it` uses stage and slot it % S:
+  // one release (the slot's) frees both
+  constexpr bool kJoint = (S == A);
   constexpr int CH = BT < 32 ? BT : 32;  // accumulator columns per TMEM load
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -274,6 +278,8 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float* amx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(wfull) + 512);  // FQ: [CS][16]
   float* sxs = amx + 8 * 16;                                                       // FQ: s_x [16]
+  // blocks each expansion warp has reported ready (a hint for the MMA warp)
+  volatile int* prog = reinterpret_cast<volatile int*>(reinterpret_cast<uint8_t*>(wfull) + 1088);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -301,6 +307,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     if (FQ) mbar_arrive_expect_tx(amaxbar, (uint32_t)(CS - 1) * 16 * 4);
     *abort_flag = 0;
     *last_flag = 0;
+    for (int e = 0; e < 4; ++e) prog[e] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
@@ -385,7 +392,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       int stage = P % S;
       uint32_t phase = (uint32_t)(P / S) & 1u;
       for (int it = P; it < total; ++it, cw.next(KB, p.tiles_m)) {
-        if (!lane0_wait(&empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
+        if (!lane0_wait(kJoint ? &aempty[stage] : &empty[stage], phase ^ 1u, abort_flag)) goto producer_done;
         if (leader) {
           const int kb = cw.kb, tile_m = cw.tile_m, tile_n = cw.tile_n;
           uint8_t* wb = wring + stage * C::kWStage;
@@ -426,10 +433,12 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
     // ---------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = idesc_i8(BT);
     // A wait costs about as much as a K-block of small MMAs, so the loop waits
-    // as little as it can: once for all the preloaded activation tiles; on the
-    // weight side, expansion finishes K-blocks in order, so a completed later
-    // block covers every block before it.  Stages and slots are released only
-    // when a later K-block will reuse them.
+    // as little as it can: once for all the preloaded activation tiles; the
+    // activation tiles of later blocks are waited for by the expansion warps,
+    // so that a completed slot means a block ready in full; expansion
+    // finishes K-blocks in order, so a completed later block covers every
+    // block before it.  Stages and slots are released only when a later
+    // K-block will reuse them.
     const int total = (int)(u_end - u_begin);
     const int P = min(S, total);
     bool any = false, x_first_seen = false;
@@ -441,27 +450,27 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
         bool ok = true;
         int run = 1;  // K-blocks from `it` on that need no further wait
         if (leader) {
-          const int stage = it % S, slot = it % A;
-          if (it < P) {
-            if (!x_first_seen) ok = mbar_wait(xfirst, 0, abort_flag);
-            x_first_seen = true;
-          } else {
-            ok = mbar_wait(&xfull[stage], (uint32_t)(it / S - 1) & 1u, abort_flag);
-          }
+          const int slot = it % A;
+          if (!x_first_seen) ok = mbar_wait(xfirst, 0, abort_flag);
+          x_first_seen = true;
           if (ok && it >= ready) {
-            ok = (ovf && it == A) ? mbar_wait(ovfull, 0, abort_flag)
-                                  : mbar_wait(&afull[slot], (uint32_t)(it / A) & 1u, abort_flag);
-            ready = it + 1;
-            // inside the window of preloaded stages the expansion usually runs
-            // ahead (it works while this kernel waits for its inputs): one look
-            // at the furthest block there may cover all the blocks before it
-            const int hi = min(it + A - 1, P - 1);
-            if (ok && hi > it && (!ovf || hi < A) &&
-                mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u))
+            // The expansion usually runs ahead.  Every expansion warp reports
+            // the blocks it has handed over; the slowest report names the
+            // furthest block that is likely complete, and one look at its slot
+            // (whose previous block this warp has consumed: at most A - 1
+            // ahead) covers every block before it.
+            const int rep_ = min(min(prog[0], prog[1]), min(prog[2], prog[3]));
+            const int hi = min(min(rep_ - 1, it + A - 1), total - 1);
+            if (hi > it && (!ovf || hi < A) && mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u)) {
               ready = hi + 1;
+            } else {
+              ok = (ovf && it == A) ? mbar_wait(ovfull, 0, abort_flag)
+                                    : mbar_wait(&afull[slot], (uint32_t)(it / A) & 1u, abort_flag);
+              ready = it + 1;
+            }
             if (ok && ovf && ready == A && mbar_try_wait(smem_u32(ovfull), 0)) ready = A + 1;
           }
-          run = min(min(ready, it < P ? P : it + 1) - it, kb1 - kb);
+          run = min(ready - it, kb1 - kb);
         }
         run = __shfl_sync(0xffffffffu, ok ? run : 0, 0);
         if (run <= 0) goto mma_done;
@@ -488,7 +497,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           int r = 0;
           for (; r < r_both; ++r) {
             issue(r);
-            tc_commit(&empty[stage]);
+            if constexpr (!kJoint) tc_commit(&empty[stage]);
             tc_commit(&aempty[slot]);
             if (++stage == S) stage = 0;
             if (++slot == A) slot = 0;
@@ -654,6 +663,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       return true;
     };
     int it_e = 0;
+    const int P_e = min(S, total_e);  // blocks from P_e on are refills of a stage
     // the first block that waits for an MMA (or the end; with the overflow
     // block in shared memory no block does)
     const int x_at = ovf ? total_e : min(A, total_e);
@@ -706,8 +716,17 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           tmem_st_32x32b_x32(t_lane + C::kAccCols + slot * 32, v);
           tmem_st_wait();
           tc_fence_before();
+          // a refilled block's activation tile: one warp sees it land before
+          // the slot is reported ready (the MMA warp waits for the slot only)
+          bool x_ok = true;
+          if (warp == 2 && it_e >= P_e && lane == 0)
+            x_ok = mbar_wait(&xfull[stage], (uint32_t)(it_e / S - 1) & 1u, abort_flag);
           __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[slot]);
+          if (lane == 0 && x_ok) {
+            mbar_arrive(&afull[slot]);
+            prog[warp - 2] = it_e + 1;
+          }
+          if (!__shfl_sync(0xffffffffu, x_ok ? 1 : 0, 0)) goto epi_done;
         }
         if (++stage == S) {
           stage = 0;
