@@ -764,29 +764,35 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
         sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
       }
       // split-K clusters: the scales of the piece this thread will write (the
-      // reduce-scatter's owner phase), also loaded before the accumulator wait
+      // reduce-scatter's owner phase), also loaded before the accumulator wait.
+      // In that phase lane l takes rows 4 (l % 8) .. 4 (l % 8) + 3 of the owned
+      // quarter (16-byte reads of the staged partial sums) and token l / 8 of
+      // each group of four of the warp's tokens.
       constexpr int kWarpsPerPiece = 4 / C::kOwned;         // CS = 2: two quarters, two warps each
-      constexpr int kTok = C::kPieceT / kWarpsPerPiece;     // tokens per thread in the owner phase
-      constexpr int kTokPre = (CS >= 2 && kTok <= 8) ? kTok : 1;
+      constexpr int kTok = C::kPieceT / kWarpsPerPiece;     // tokens per warp in the owner phase
+      constexpr int kSxRegs = (kTok + 31) / 32;             // token i's scale: register i / 32 of lane i % 32
       const int oe = warp - 2;
       const int opidx = CS >= 4 ? 0 : oe % C::kOwned;
       const int oqq = CS >= 4 ? (int)crank / C::kSlices : (int)crank * C::kOwned + opidx;  // owned quarter
       const int ohh = CS >= 4 ? (int)crank % C::kSlices : 0;                               // owned token slice
       const int ot0 = CS >= 4 ? oe : oe / C::kOwned;
-      const int onn = tile_n * kBlockN + oqq * 32 + lane;
-      const bool onn_ok = onn < p.N;
-      float oscn = 0.0f;
-      float osx[kTokPre];
+      const int orow = oqq * 32 + (lane & 7) * 4;           // this lane's first row in the tile
+      const int onn = tile_n * kBlockN + orow;
+      const bool onn_ok = onn < p.N;                        // N % 16 == 0: all four rows or none
+      float osc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float osl[kSxRegs];
 #pragma unroll
-      for (int i = 0; i < kTokPre; ++i) osx[i] = 0.0f;
+      for (int j = 0; j < kSxRegs; ++j) osl[j] = 0.0f;
       if constexpr (CS >= 2 && !OUT_I32) {
-        oscn = onn_ok ? __ldg(p.s_c + onn) : 0.0f;
-        if constexpr (kTok <= 8) {
+        if (onn_ok) {
 #pragma unroll
-          for (int i = 0; i < kTok; ++i) {
-            const int m = m0 + ohh * C::kPieceT + ot0 + i * kWarpsPerPiece;
-            osx[i] = (m < p.M) ? (FQ ? sxs[m - m0] : __ldg(p.s_x + m)) : 0.0f;
-          }
+          for (int q4 = 0; q4 < 4; ++q4) osc[q4] = __ldg(p.s_c + onn + q4);
+        }
+#pragma unroll
+        for (int j = 0; j < kSxRegs; ++j) {
+          const int i = j * 32 + lane;
+          const int m = m0 + ohh * C::kPieceT + ot0 + i * kWarpsPerPiece;
+          osl[j] = (i < kTok && m < p.M) ? (FQ ? sxs[m - m0] : __ldg(p.s_x + m)) : 0.0f;
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
@@ -849,23 +855,55 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           red_done = true;
           {
             const uint32_t* own = reinterpret_cast<const uint32_t*>(xring) + (size_t)oqq * BT * 32 + (size_t)ohh * T * 32;
-#pragma unroll 4
-            for (int i = 0; i < kTok; ++i) {
-              const int t = ot0 + i * kWarpsPerPiece;  // token within the piece
-              const int m = m0 + ohh * T + t;
-              uint32_t acc = own[t * 32 + lane];
+            const uint32_t* rsrc = reinterpret_cast<const uint32_t*>(red) + (size_t)opidx * T * 32;
+            const int tsub = lane >> 3;  // token of the group of four
+            const int rcol = (lane & 7) * 4;
+            // two groups (8 tokens) per step: all their partial sums are read
+            // before any of their stores (a store may not be moved above a
+            // later load of shared memory the compiler cannot tell apart from it)
+            constexpr int kGroups = (kTok + 3) / 4;
+            constexpr int kGC = kGroups < 2 ? kGroups : 2;
+#pragma unroll 1
+            for (int g0 = 0; g0 < kGroups; g0 += kGC) {
+              uint4 acc[kGC];
+              int tk[kGC];
 #pragma unroll
-              for (int sidx = 0; sidx < CS - 1; ++sidx)
-                acc += (uint32_t)red[((size_t)sidx * C::kOwned + opidx) * T * 32 + t * 32 + lane];
-              if (m < p.M && onn_ok) {
-                if constexpr (OUT_I32) {
-                  reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + onn] = (int32_t)acc;
-                } else {
-                  float sxm;
-                  if constexpr (kTok <= 8) sxm = osx[i];
-                  else sxm = FQ ? sxs[m - m0] : __ldg(p.s_x + m);
-                  const float y = __fmul_rn(__int2float_rn((int32_t)acc), __fmul_rn(sxm, oscn));
-                  reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + onn] = __float2bfloat16_rn(y);
+              for (int c = 0; c < kGC; ++c) {
+                const int i = (g0 + c) * 4 + tsub;  // this lane's token among the warp's
+                tk[c] = ot0 + (i < kTok ? i : 0) * kWarpsPerPiece;  // token within the piece
+                acc[c] = *reinterpret_cast<const uint4*>(own + tk[c] * 32 + rcol);
+#pragma unroll
+                for (int sidx = 0; sidx < CS - 1; ++sidx) {
+                  const uint4 v = *reinterpret_cast<const uint4*>(rsrc + (size_t)sidx * C::kOwned * T * 32 + tk[c] * 32 + rcol);
+                  acc[c].x += v.x;
+                  acc[c].y += v.y;
+                  acc[c].z += v.z;
+                  acc[c].w += v.w;
+                }
+              }
+#pragma unroll
+              for (int c = 0; c < kGC; ++c) {
+                const int i = (g0 + c) * 4 + tsub;
+                const int m = m0 + ohh * T + tk[c];
+                // the token's scale, already in registers (lane-distributed)
+                float sxm = 0.0f;
+                if constexpr (!OUT_I32)
+                  sxm = __shfl_sync(0xffffffffu, (kSxRegs == 1 || (g0 + c) * 4 < 32) ? osl[0] : osl[kSxRegs - 1], i & 31);
+                if (i < kTok && m < p.M && onn_ok) {
+                  if constexpr (OUT_I32) {
+                    *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.out) + (size_t)m * p.N + onn) = acc[c];
+                  } else {
+                    const uint32_t av[4] = {acc[c].x, acc[c].y, acc[c].z, acc[c].w};
+                    uint32_t h[2];
+#pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                      const float y0 = __fmul_rn(__int2float_rn((int32_t)av[2 * q2]), __fmul_rn(sxm, osc[2 * q2]));
+                      const float y1 = __fmul_rn(__int2float_rn((int32_t)av[2 * q2 + 1]), __fmul_rn(sxm, osc[2 * q2 + 1]));
+                      const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                      h[q2] = *reinterpret_cast<const uint32_t*>(&b2);
+                    }
+                    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.N + onn) = make_uint2(h[0], h[1]);
+                  }
                 }
               }
             }
