@@ -150,16 +150,38 @@ int stages_of(int bt) {
   }
 }
 
+// whether two CTAs of the tile kernel fit one SM (shared memory and TMEM)
+template <int BT, int CS>
+bool fits_two_t() {
+  using C = lq::GemmCfg<BT, CS>;
+  return C::kTmemCols <= 256 && 2 * (C::kSmemBytes + 1024) <= 233472;
+}
+bool fits_two_per_sm(int bt, int cs) {
+  switch (bt * 16 + cs) {
+    case 16 * 16 + 2: return fits_two_t<16, 2>();
+    case 16 * 16 + 4: return fits_two_t<16, 4>();
+    case 16 * 16 + 8: return fits_two_t<16, 8>();
+    case 32 * 16 + 2: return fits_two_t<32, 2>();
+    case 32 * 16 + 4: return fits_two_t<32, 4>();
+    case 32 * 16 + 8: return fits_two_t<32, 8>();
+    case 64 * 16 + 2: return fits_two_t<64, 2>();
+    case 64 * 16 + 4: return fits_two_t<64, 4>();
+  }
+  return false;
+}
+
 Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms) {
   Schedule s;
   int kind = schedule;
   int bt = block_t ? block_t : auto_block_t(M);
   if (kind == kSchedAuto) {
-    // enough 256 x 256 tiles to give every CTA pair one: CTA pairs; many tiles
-    // of 128 tokens: persistent; otherwise one cluster per tile
+    // enough 256 x 256 tiles for half of the CTA pairs: CTA pairs (a pair
+    // kernel tile costs about as much SM time as two 128-token tiles of the
+    // persistent kernel, so it wins even when some pairs stay idle); many
+    // tiles of 128 tokens: persistent; otherwise one cluster per tile
     const long long t128 = (long long)((M + lq::kPBT - 1) / lq::kPBT) * ((N + lq::kBlockN - 1) / lq::kBlockN);
     const long long t256 = (long long)((M + lq::kQBT - 1) / lq::kQBT) * ((N + lq::kQBN - 1) / lq::kQBN);
-    if (block_t == 0 && K % lq::kQBK == 0 && t256 >= sms / 2)
+    if (block_t == 0 && K % lq::kQBK == 0 && t256 >= sms / 4)
       kind = kSchedPair;
     else
       kind = (bt == lq::kPBT && t128 >= sms) ? kSchedPersistent : kSchedTiles;
@@ -223,11 +245,11 @@ Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split
         break;
       }
     // When a CTA's K-slice is longer than its preloaded stages, the ring
-    // streams the rest anyway and more CTAs stream faster: tiles of up to 64
-    // tokens fit two CTAs per SM (256 TMEM columns), so use that capacity.
+    // streams the rest anyway and more CTAs stream faster: where two CTAs of
+    // a wider split fit one SM, use that capacity.
     if (s.KB / cs > stages_of(s.bt) && s.bt <= 64)
       for (int c = max_split(s.bt); c > cs; c /= 2)
-        if (s.tiles * c <= 2LL * sms && s.KB / c >= 4) {
+        if (fits_two_per_sm(s.bt, c) && s.tiles * c <= 2LL * sms && s.KB / c >= 4) {
           cs = c;
           break;
         }
