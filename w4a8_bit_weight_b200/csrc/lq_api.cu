@@ -175,13 +175,14 @@ Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split
   int kind = schedule;
   int bt = block_t ? block_t : auto_block_t(M);
   if (kind == kSchedAuto) {
-    // enough 256 x 256 tiles for half of the CTA pairs: CTA pairs (a pair
-    // kernel tile costs about as much SM time as two 128-token tiles of the
-    // persistent kernel, so it wins even when some pairs stay idle); many
-    // tiles of 128 tokens: persistent; otherwise one cluster per tile
+    // more than 128 tokens and enough 256 x 256 tiles for half of the CTA
+    // pairs: CTA pairs (a pair kernel tile costs about as much SM time as two
+    // 128-token tiles of the persistent kernel, so it wins even when some
+    // pairs stay idle); many tiles of 128 tokens: persistent; otherwise one
+    // cluster per tile
     const long long t128 = (long long)((M + lq::kPBT - 1) / lq::kPBT) * ((N + lq::kBlockN - 1) / lq::kBlockN);
     const long long t256 = (long long)((M + lq::kQBT - 1) / lq::kQBT) * ((N + lq::kQBN - 1) / lq::kQBN);
-    if (block_t == 0 && K % lq::kQBK == 0 && t256 >= sms / 4)
+    if (block_t == 0 && K % lq::kQBK == 0 && M > lq::kPBT && t256 >= sms / 4)
       kind = kSchedPair;
     else
       kind = (bt == lq::kPBT && t128 >= sms) ? kSchedPersistent : kSchedTiles;
