@@ -130,6 +130,8 @@ SHAPES = [
     (300, 272, 1024, 0, PR, 0, 0),        # CTA pairs: ragged M and N
     (512, 512, 2048, 0, PR, 0, 2),        # one pair, four tiles: accumulator handed back and forth
     (1000, 768, 768, 0, PR, 0, 4),        # two pairs, 12 tiles, ragged M
+    (512, 512, 1024, 0, PR, 0, 6),        # 4 tiles over 3 pairs: the last tile in token halves
+    (700, 512, 512, 0, PR, 0, 10),        # 6 tiles over 5 pairs: ragged M in the split last tile
     (16, 256, 1024, 16, SK, 0, 2),        # stream-K, one CTA per tile
     (16, 256, 1024, 16, SK, 0, 3),        # stream-K: split tiles through the workspace
     (16, 256, 1024, 16, SK, 0, 16),       # one K-block per CTA

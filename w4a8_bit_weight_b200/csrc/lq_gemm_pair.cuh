@@ -21,6 +21,9 @@
 // the epilogue warps of both CTAs hand it back as soon as it sits in their
 // registers as packed bf16, before any global store.
 //
+// When the tiles leave the last round at most half full, that round's tiles
+// are cut into halves of 128 tokens (N = 128 MMAs), one half per pair.
+//
 // Activation stage i and TMEM weight slot i are filled and drained together,
 // so one barrier pair covers both.  Hand-offs between the two CTAs:
 //   activations landed   -> both CTAs' activation copies complete their bytes on
@@ -104,9 +107,28 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_ma
       "h"(cta_mask)
       : "memory");
 }
-__device__ __forceinline__ uint32_t idesc_i8_pair() {
-  return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kQBT >> 3) << 17) | (uint32_t(kQBN >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_i8_pair(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kQBN >> 4) << 24);
 }
+
+// A pair's share of the tiles: whole tiles cid, cid + ncl, ...  When the last
+// round would leave at least half of the pairs idle, its tiles are cut into
+// token halves instead (an N = 128 pair MMA costs half an N = 256 one), one
+// half per pair, so that round takes half as long.
+struct PairWork {
+  int nwhole, nunits, tail_tile, tail_half;
+  __device__ __forceinline__ PairWork(int cid, int ncl, int tiles) {
+    const int rounds = tiles / ncl, rem = tiles - rounds * ncl;
+    const bool split = rem > 0 && 2 * rem <= ncl;
+    nwhole = split ? rounds : (cid < tiles ? (tiles - 1 - cid) / ncl + 1 : 0);
+    nunits = nwhole + ((split && cid < 2 * rem) ? 1 : 0);
+    tail_tile = rounds * ncl + (cid >> 1);
+    tail_half = cid & 1;
+  }
+  __device__ __forceinline__ int tile(int k, int cid, int ncl) const { return k < nwhole ? cid + k * ncl : tail_tile; }
+  // -1: the whole tile; 0 / 1: that half of its 256 tokens
+  __device__ __forceinline__ int half(int k) const { return k < nwhole ? -1 : tail_half; }
+};
 
 // Arrive on the even CTA's copy of `bar` (local arrive on the even CTA).
 __device__ __forceinline__ void arrive_on_leader(uint64_t* bar, uint32_t crank) {
@@ -197,9 +219,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int tiles = (int)(p.U);             // host passes the tile count in U
   const int cid = blockIdx.x >> 1;
   const int ncl = gridDim.x >> 1;
-  int ntiles = 0;
-  for (int tile = cid; tile < tiles; tile += ncl) ++ntiles;
-  const int total = ntiles * KS;            // K-blocks this CTA takes part in
+  const PairWork pw(cid, ncl, tiles);
+  const int total = pw.nunits * KS;         // K-blocks this CTA takes part in
 
   if (warp == 0) {
     // ---------------------------------------------------- weight producer
@@ -208,7 +229,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
     if (leader) pol = l2_policy_evict_first();
     uint32_t issued = 0, issued_par = 0;
     int it = 0;
-    for (int tile = cid; tile < tiles; tile += ncl) {
+    for (int k = 0; k < pw.nunits; ++k) {
+      const int tile = pw.tile(k, cid, ncl);
       const int wrow = (tile / tiles_m) * kQBN + (int)crank * 128;
       for (int kb = 0; kb < KS; ++kb, ++it) {
         const int w = it % SW;
@@ -241,8 +263,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const uint32_t full_even = mapa_shared(smem_u32(full), 0);
     bool issued = false;
     int it = 0;
-    for (int tile = cid; tile < tiles; tile += ncl) {
-      const int xrow = (tile % tiles_m) * kQBT + (int)crank * 128;
+    for (int k = 0; k < pw.nunits; ++k) {
+      const int tile = pw.tile(k, cid, ncl), half = pw.half(k);
+      // B is split by N across the pair: 128 tokens per CTA, 64 for a half tile
+      // (the 128-row box then carries 64 rows the MMA does not read)
+      const int xrow = (tile % tiles_m) * kQBT + (half < 0 ? (int)crank * 128 : half * 128 + (int)crank * 64);
       for (int kb = 0; kb < KS; ++kb, ++it) {
         const int x = it % SX;
         const uint32_t use = (uint32_t)(it / SX);
@@ -269,10 +294,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
   } else if (warp == 1) {
     if (even) {
       // ------------------------------------------------- MMA issuer (even CTA)
-      const uint32_t idesc = idesc_i8_pair();
       bool any = false;
       int it = 0, j = 0;
-      for (int tile = cid; tile < tiles; tile += ncl, ++j) {
+      for (int k = 0; k < pw.nunits; ++k, ++j) {
+        const uint32_t idesc = idesc_i8_pair(pw.half(k) < 0 ? kQBT : kQBT / 2);
         // the single accumulator is free once both CTAs' epilogues have loaded it
         if (!warp_wait(accempty, ((uint32_t)j & 1u) ^ 1u, abort_flag, true)) goto mma_done;
         tc_fence_after();
@@ -358,11 +383,22 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     griddep_wait();
     int j = 0;
-    for (int tile = cid; tile < tiles; tile += ncl, ++j) {
+    for (int k = 0; k < pw.nunits; ++k, ++j) {
+      const int tile = pw.tile(k, cid, ncl), half = pw.half(k);
       const int tm = tile % tiles_m, tn = tile / tiles_m;
       const int n = tn * kQBN + (int)crank * 128 + r;
       const bool n_ok = n < p.N;
-      const int mb = tm * kQBT + e * 128;
+      // a half tile's 128 tokens are accumulator columns 0-127: the second
+      // pair of warps only hands the accumulator back
+      const int mb = tm * kQBT + (half < 0 ? e * 128 : half * 128);
+      if (half >= 0 && e == 1) {
+        if (!warp_wait(accfull, (uint32_t)j & 1u, abort_flag, false)) goto epi_done;
+        tc_fence_after();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(accempty, crank);
+        continue;
+      }
       // scales are loaded before the accumulator is ready, off the hand-back path
       const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
       float sx4[4];  // s_x of tokens mb + 32c + lane
