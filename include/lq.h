@@ -270,6 +270,47 @@ LQ_API lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const
                                       void* out_bf16, int M, int N, int K, int group, void* stream);
 
 /*
+ * lq_w4a8_grouped_gemm -- the W4A8 GEMM for a mixture-of-experts layer (one
+ * weight matrix per group, or expert, each applied to its own run of token
+ * rows): out[m, n] = bf16((sum_k x_q[m,k] * Q_hat[e*N + n, k]) * s_x[m] *
+ * s_c[e*N + n]) for the rows m in [m_off[e], m_off[e+1]) of group e.  The
+ * models the review page names for the accuracy study include the
+ * mixture-of-experts Mixtral-8x7B ("What would settle it"); the grouped form
+ * is this library's, not the paper's.
+ *   x_q, s_x: [M, K] int8 and [M] fp32 from lq_quantize_act, the rows of
+ *     each group contiguous and in group order (a router's sorted token
+ *     copies).
+ *   qw, s_u8, a_u8, s_c: the `groups` weight matrices stacked as one
+ *     [groups * N, K] matrix and quantized in one lq_quantize_weights call
+ *     (quantization is per row, so stacking changes nothing).
+ *   m_off: DEVICE int32 [groups + 1], non-decreasing, m_off[0] = 0,
+ *     m_off[groups] = M; it may be written by the kernel that precedes this
+ *     one on the stream (it is read after the grid dependency wait).
+ *     Empty groups are allowed.  Offsets that break these rules give
+ *     undefined (but in-bounds) results.
+ *   out_bf16: [M, N] bf16, row m for the group that owns m.
+ *   Requires N % 128 == 0 (a weight tile never spans two groups), the GEMM's
+ *   K and group rules, 1 <= groups <= LQ_MAX_GROUPS, 16-byte-aligned
+ *   x_q, qw, s_u8, a_u8, out and 4-byte-aligned s_x, s_c, m_off.  No
+ *   workspace.  One thread-block cluster per 128-row weight tile and token
+ *   tile (split-K inside the cluster for small token counts); clusters whose
+ *   token tile lies past the last group's rows exit at once.
+ * lq_w4a8_grouped_gemm_ex adds block_t (0 = from the mean rows per group,
+ *   else 16, 32, 64 or 128), split_k (0 = automatic, else as in
+ *   LQ_SCHED_TILES) and out_i32 (int32 accumulators to `out`, s_x and s_c
+ *   unused).
+ */
+#define LQ_MAX_GROUPS 1024
+LQ_API lq_status lq_w4a8_grouped_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                                      const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c,
+                                      const int* m_off, int groups, void* out_bf16, int M, int N, int K,
+                                      int group, void* stream);
+LQ_API lq_status lq_w4a8_grouped_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                                         const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c,
+                                         const int* m_off, int groups, void* out, int M, int N, int K,
+                                         int group, int block_t, int split_k, int out_i32, void* stream);
+
+/*
  * lq_get_device_error -- synchronizes `stream`, then reads and clears the
  * library's device error word.  Returns LQ_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last call (its output is then undefined),

@@ -236,3 +236,25 @@ def w4a8_gemm_sampled(x_q, s_x, qw, s_u8, a_u8, s_c, m_idx, n_idx, group: int = 
                                                _p(s_c), M, N, K, group, _p(m_idx), _p(n_idx), cnt,
                                                _p(out), _p(acc)), "w4a8_gemm_sampled")
     return out, acc
+
+
+def w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N: int, group: int = GROUP):
+    """Grouped GEMM (one weight matrix per group, e.g. the experts of a
+    mixture-of-experts layer): token rows [m_off[e], m_off[e+1]) of x_q times
+    weight rows [e*N, (e+1)*N) of the stacked quantized weights, written out
+    as one w4a8_gemm per group.  Returns (out uint16 [M,N], acc int32 [M,N])."""
+    x_q = np.ascontiguousarray(x_q, np.int8)
+    m_off = [int(v) for v in m_off]
+    M, K = x_q.shape
+    out = np.zeros((M, N), np.uint16)
+    acc = np.zeros((M, N), np.int32)
+    for e in range(len(m_off) - 1):
+        r0, r1 = m_off[e], m_off[e + 1]
+        if r1 <= r0:
+            continue
+        o, a = w4a8_gemm(x_q[r0:r1], np.asarray(s_x)[r0:r1], np.asarray(qw)[e * N:(e + 1) * N],
+                         np.asarray(s_u8)[:, e * N:(e + 1) * N], np.asarray(a_u8)[:, e * N:(e + 1) * N],
+                         np.asarray(s_c)[e * N:(e + 1) * N], group)
+        out[r0:r1] = o
+        acc[r0:r1] = a
+    return out, acc

@@ -140,3 +140,22 @@ def test_linear_workspace_size_rules(lib):
     assert w(16, 4096, 14336) == 16 * 14336 + 64
     assert w(16, 200, 512) == 0   # invalid shape
     assert wx(16, 4096, 4096, 5) == 0  # invalid path
+
+
+def test_grouped_rejects_before_launch(lib):
+    f = lib.lq_w4a8_grouped_gemm_ex
+
+    def call(M=32, N=256, K=512, group=64, groups=4, x=GOOD, sx=GOOD, qw=GOOD, s=GOOD, a=GOOD, sc=GOOD,
+             off=GOOD, out=GOOD, bt=0, split=0, i32=0):
+        return f(x, sx, qw, s, a, sc, off, groups, out, M, N, K, group, bt, split, i32, None)
+
+    assert call(N=192) == 2                  # a weight tile would span two groups
+    assert call(N=200) == 2 and call(K=192) == 2 and call(group=32) == 2
+    assert call(groups=0) == 1 and call(groups=lq.MAX_GROUPS + 1) == 1
+    assert call(bt=256) == 1 and call(bt=48) == 1 and call(split=-1) == 1
+    assert call(bt=64, split=8) == 1         # split 8 only for tiles of <= 32 tokens
+    assert call(off=P(0)) == 1 and call(x=P(0)) == 1 and call(sc=P(0)) == 1
+    assert call(i32=1, sc=P(0), sx=P(0)) != 1  # the int32 form takes no scales (then needs a device)
+    assert call(x=ODD) == 3 and call(out=ODD) == 3 and call(off=P((1 << 20) + 2)) == 3
+    assert call(M=0) == 0                    # empty batch: nothing to launch
+    assert call(M=-1) == 1

@@ -349,3 +349,31 @@ def test_sampled_equals_full():
     so, sa = oracle.w4a8_gemm_sampled(x_q, s_x, qw, s_u8, a_u8, s_c, mi.ravel(), ni.ravel())
     np.testing.assert_array_equal(so, out.ravel())
     np.testing.assert_array_equal(sa, acc.ravel())
+
+
+# ---------------------------------------------------------------------------
+# Grouped GEMM (one weight matrix per group): against a float64 product of the
+# dequantized stacked weights, each row taking the columns of its own group
+# ---------------------------------------------------------------------------
+
+def test_grouped_gemm_against_float64_rows():
+    from w4a8_bit_weight_b200 import synth
+    E, N, K = 4, 32, 256
+    m_off = [0, 3, 3, 10, 13]          # group 1 is empty
+    M = m_off[-1]
+    X, W = synth.make_problem(M, E * N, K, seed=41, n_outliers=2)
+    qw, s_u8, a_u8, s_c, _ = oracle.quantize_weights(synth.bf16_bits(W))
+    x_q, s_x = oracle.quantize_act(synth.bf16_bits(X))
+    out, acc = oracle.w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N)
+    w_hat = oracle.dequant(qw, s_u8, a_u8).astype(np.float64)          # [E*N, K]
+    full = x_q.astype(np.float64) @ w_hat.T                               # [M, E*N]
+    for e in range(E):
+        for m in range(m_off[e], m_off[e + 1]):
+            np.testing.assert_array_equal(acc[m].astype(np.float64), full[m, e * N:(e + 1) * N])
+            ref = oracle.epilogue(acc[m:m + 1], s_x[m:m + 1], s_c[e * N:(e + 1) * N])
+            np.testing.assert_array_equal(out[m], ref[0])
+    # one group is the plain GEMM
+    o1, a1 = oracle.w4a8_grouped_gemm(x_q, s_x, qw[:N], s_u8[:, :N], a_u8[:, :N], s_c[:N], [0, M], N)
+    o2, a2 = oracle.w4a8_gemm(x_q, s_x, qw[:N], s_u8[:, :N], a_u8[:, :N], s_c[:N])
+    np.testing.assert_array_equal(a1, a2)
+    np.testing.assert_array_equal(o1, o2)

@@ -26,6 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblq_b200.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lq.h")
 GROUP = 64
+MAX_GROUPS = 1024  # LQ_MAX_GROUPS in lq.h
 SCHED_AUTO, SCHED_TILES, SCHED_PERSISTENT, SCHED_STREAMK, SCHED_PAIR = 0, 1, 2, 3, 4
 
 STATUS = {
@@ -74,6 +75,8 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_linear": ([P, P, P, P, P, P, I, I, I, I, P, Z, P], I),
             "lq_w4a8_linear_workspace_size_ex": ([I, I, I, I], Z),
             "lq_w4a8_linear_ex": ([P, P, P, P, P, P, I, I, I, I, P, Z, I, P], I),
+            "lq_w4a8_grouped_gemm": ([P, P, P, P, P, P, P, I, P, I, I, I, I, P], I),
+            "lq_w4a8_grouped_gemm_ex": ([P, P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -296,6 +299,36 @@ def lq_w4a8_gemm_noalloc(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = G
         _check("lq_w4a8_gemm_noalloc", lib.lq_w4a8_gemm_noalloc(
             _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out),
             M, N, K, group, _stream(x_q.device)))
+    return out
+
+
+def lq_w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N: int, out=None, group: int = GROUP,
+                         block_t: int = 0, split_k: int = 0, out_i32: bool = False):
+    """Grouped W4A8 GEMM (mixture-of-experts layer): rows [m_off[e], m_off[e+1]) of x_q times
+    weight rows [e*N, (e+1)*N) of the stacked quantized weights -> [M, N] bf16 (int32 with out_i32).
+
+    m_off is a device int32 tensor of groups + 1 non-decreasing row offsets (0 ... M)."""
+    lib = load_library()
+    _need(x_q, torch.int8, "x_q")
+    M, K = x_q.shape
+    _need(m_off, torch.int32, "m_off")
+    if m_off.dim() != 1 or m_off.numel() < 2:
+        raise ValueError("m_off must hold groups + 1 >= 2 offsets")
+    G = m_off.numel() - 1
+    _need(qw, torch.uint8, "qw", (G * N, K // 2))
+    _need(s_u8, torch.uint8, "s_u8", (K // group, G * N))
+    _need(a_u8, torch.uint8, "a_u8", (K // group, G * N))
+    if not out_i32:
+        _need(s_x, torch.float32, "s_x", (M,))
+        _need(s_c, torch.float32, "s_c", (G * N,))
+    odt = torch.int32 if out_i32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(M, N, dtype=odt, device=x_q.device)
+    _need(out, odt, "out", (M, N))
+    with torch.cuda.device(x_q.device):
+        _check("lq_w4a8_grouped_gemm", lib.lq_w4a8_grouped_gemm_ex(
+            _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(m_off), G, _ptr(out),
+            M, N, K, group, block_t, split_k, 1 if out_i32 else 0, _stream(x_q.device)))
     return out
 
 

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <cstdlib>
@@ -716,6 +717,89 @@ lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const uint8_
     return LQ_ERR_CUDA;
   return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, scratch, kNoAllocScratchBytes, 0,
                    kSchedStreamK, 0, 0, false, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ grouped GEMM
+// Mixture-of-experts layers: every group (expert) has its own N x K weights,
+// stacked as one [groups * N, K] matrix quantized in one call, and its own
+// contiguous run of token rows.  One cluster per tile, as in the tile
+// schedule; the token tiles of all groups are enumerated from a bound that
+// needs no device data, and each cluster finds its group from the row
+// offsets on the device.
+namespace {
+
+lq_status grouped_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                       const uint8_t* a_u8, const float* s_c, const int* m_off, int groups, void* out, int M, int N,
+                       int K, int group, int block_t, int split_k, bool out_i32, void* stream) {
+  lq_status st = check_gemm_shape(M, N, K, group);
+  if (st != LQ_OK) return st;
+  if (N % lq::kBlockN != 0) return LQ_ERR_UNSUPPORTED_SHAPE;  // a weight tile never spans two groups
+  if (groups < 1 || groups > LQ_MAX_GROUPS || (long long)groups * N > INT_MAX) return LQ_ERR_INVALID_ARG;
+  if (block_t != 0 && (block_t == 256 || !valid_block_t(block_t))) return LQ_ERR_INVALID_ARG;
+  if (split_k < 0) return LQ_ERR_INVALID_ARG;
+  if (M == 0) return LQ_OK;
+  if (!x_q || !qw || !s_u8 || !a_u8 || !out || !m_off || (!out_i32 && (!s_x || !s_c))) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x_q, 16) || !aligned(qw, 16) || !aligned(s_u8, 16) || !aligned(a_u8, 16) || !aligned(out, 16) ||
+      !aligned(m_off, 4) || (s_x && !aligned(s_x, 4)) || (s_c && !aligned(s_c, 4)))
+    return LQ_ERR_MISALIGNED;
+  // token tile from the mean rows per group; the token tiles of all groups
+  // number at most sum(ceil(M_e / bt)) <= (M + groups (bt - 1)) / bt, and at most M
+  const int bt = block_t ? block_t : auto_block_t((M + groups - 1) / groups);
+  if (split_k > 0 && !valid_split(bt, split_k)) return LQ_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  const long long tm_bound = std::min<long long>(((long long)M + (long long)groups * (bt - 1)) / bt, M);
+  if (tm_bound * bt > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
+  const Schedule s = make_schedule((int)(tm_bound * bt), N, K, bt, kSchedTiles, split_k, 0, dev->sms);
+  const int NT = groups * N;
+  CUtensorMap tx, tw, ts, ta;
+  if (!make_map_u8(&tx, x_q, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, (uint32_t)bt,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)NT, (uint64_t)K / 2, lq::kBlockK / 2, lq::kBlockN,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_u8(&ts, s_u8, (uint64_t)NT, (uint64_t)K / LQ_GROUP, (uint64_t)NT, lq::kBlockN, 2u,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_u8(&ta, a_u8, (uint64_t)NT, (uint64_t)K / LQ_GROUP, (uint64_t)NT, lq::kBlockN, 2u,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return LQ_ERR_CUDA;
+  lq::GemmArgs a;
+  a.x_bf16 = nullptr;
+  a.s_x = s_x;
+  a.s_c = s_c;
+  a.out = out;
+  a.ws = nullptr;
+  a.ticket = nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = s.tiles_m;
+  a.KB = s.KB;
+  a.U = s.U;
+  a.m_off = m_off;
+  a.groups = groups;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  return out_i32 ? launch_gemm<true>(s, tx, tw, ts, ta, a, cs) : launch_gemm<false>(s, tx, tw, ts, ta, a, cs);
+}
+
+}  // namespace
+
+extern "C" {
+
+lq_status lq_w4a8_grouped_gemm_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                                  const uint8_t* a_u8, const float* s_c, const int* m_off, int groups, void* out,
+                                  int M, int N, int K, int group, int block_t, int split_k, int out_i32,
+                                  void* stream) {
+  return grouped_impl(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, groups, out, M, N, K, group, block_t, split_k,
+                      out_i32 != 0, stream);
+}
+
+lq_status lq_w4a8_grouped_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                               const uint8_t* a_u8, const float* s_c, const int* m_off, int groups, void* out_bf16,
+                               int M, int N, int K, int group, void* stream) {
+  return grouped_impl(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, groups, out_bf16, M, N, K, group, 0, 0, false, stream);
 }
 
 }  // extern "C"

@@ -116,6 +116,11 @@ struct GemmArgs {
   int M, N, K;
   int tiles_m, KB;
   long long U;           // units = tiles * KB
+  // grouped GEMM (one tile per cluster): group e multiplies token rows
+  // [m_off[e], m_off[e+1]) by weight rows [e*N, (e+1)*N); tiles_m then bounds
+  // the token tiles of all groups together
+  const int* m_off = nullptr;
+  int groups = 0;
 };
 
 // (tile, K-block) of a unit, stepped without divisions: an integer division
@@ -180,13 +185,13 @@ __device__ __forceinline__ uint32_t quant_quad_i8(uint32_t w01, uint32_t w23, fl
 // < TC).  The token scales are gathered first, so that the stores do not wait
 // on one another.  Every lane of the warp must call it.
 template <bool OUT_I32, int TC>
-__device__ __forceinline__ void store_chunk(const GemmArgs& p, int m_first, int n, bool n_ok, const uint32_t* v,
+__device__ __forceinline__ void store_chunk(const GemmArgs& p, int m_first, int mend, int n, bool n_ok, const uint32_t* v,
                                             float sx_lane, float sc) {
   float scale[TC];
 #pragma unroll
   for (int i = 0; i < TC; ++i) scale[i] = __fmul_rn(__shfl_sync(0xffffffffu, sx_lane, i), sc);
   if (!n_ok) return;
-  const int mlim = p.M - m_first;
+  const int mlim = mend - m_first;
   if constexpr (OUT_I32) {
     int32_t* o = reinterpret_cast<int32_t*>(p.out) + (size_t)m_first * p.N + n;
 #pragma unroll
@@ -287,6 +292,49 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   const int lane = threadIdx.x & 31;
   const uint32_t crank = CS >= 2 ? cluster_ctarank() : 0u;
 
+  // Grouped GEMM: this cluster's tile (token tile j over all groups, weight
+  // tile tn of its group).  The row offsets may come from the preceding
+  // kernel, so the dependency wait comes first.  Every warp finds the group
+  // itself (a scan of the groups' tile counts); a tile past the last group's
+  // rows leaves at once, before any barrier, in every CTA of its cluster.
+  int g_xrow = 0, g_mend = p.M, g_wrow = 0, g_scoff = 0;
+  if (p.m_off != nullptr) {
+    griddep_wait();
+    const int t = (int)(blockIdx.x / (CS >= 1 ? CS : 1));
+    const int j = t % p.tiles_m, tn = t / p.tiles_m;
+    // offsets are read clamped to [0, M]: whatever they hold, no row outside
+    // the activations and the output is ever written
+    auto off_at = [&](int e) { return min(max(__ldg(p.m_off + e), 0), p.M); };
+    int ge = -1, before = 0, run = 0;
+    for (int base = 0; base < p.groups && ge < 0; base += 32) {
+      const int e = base + lane;
+      int cnt = 0;
+      if (e < p.groups) cnt = max(0, off_at(e + 1) - off_at(e) + BT - 1) / BT;
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && j >= run + incl - cnt && j < run + incl);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        ge = base + l;
+        before = run + __shfl_sync(0xffffffffu, incl - cnt, l);
+      }
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (ge < 0) return;
+    g_xrow = off_at(ge) + (j - before) * BT;
+    g_mend = off_at(ge + 1);
+    g_wrow = ge * p.N + tn * kBlockN;
+    g_scoff = ge * p.N;
+  }
+  const bool grouped = (p.m_off != nullptr);
+  // first token row of token tile tm, first (stacked) weight row of weight tile tn
+  auto xrow_of = [&](int tm) { return grouped ? g_xrow : tm * BT; };
+  auto wrow_of = [&](int tn) { return grouped ? g_wrow : tn * kBlockN; };
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&wfull[s], 1);
@@ -374,9 +422,10 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       if (leader) {
         uint8_t* wb = wring + i * C::kWStage;
         mbar_arrive_expect_tx(&wfull[i], C::kTxW);
-        tma_load_2d(wb, &tm_w, &wfull[i], cw.kb * (kBlockK / 2), cw.tile_n * kBlockN, pol_stream);
-        tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], cw.tile_n * kBlockN, cw.kb * 2, pol_stream);
-        tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], cw.tile_n * kBlockN, cw.kb * 2, pol_stream);
+        const int wr = wrow_of(cw.tile_n);
+        tma_load_2d(wb, &tm_w, &wfull[i], cw.kb * (kBlockK / 2), wr, pol_stream);
+        tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], wr, cw.kb * 2, pol_stream);
+        tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], wr, cw.kb * 2, pol_stream);
       }
     }
     griddep_wait();
@@ -385,7 +434,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       mbar_arrive_expect_tx(xfirst, (uint32_t)P * C::kTxX);
       UnitCursor cx = first;
       for (int i = 0; i < P; ++i, cx.next(KB, p.tiles_m))
-        tma_load_2d(xring + i * C::kXBytes, &tm_x, xfirst, cx.kb * kBlockK, cx.tile_m * BT, pol_keep);
+        tma_load_2d(xring + i * C::kXBytes, &tm_x, xfirst, cx.kb * kBlockK, xrow_of(cx.tile_m), pol_keep);
     }
     __syncwarp();
     // xfull[s] serves the refills of stage s only: its k-th phase is the (k+1)-th use of the stage
@@ -399,11 +448,12 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           const int kb = cw.kb, tile_m = cw.tile_m, tile_n = cw.tile_n;
           uint8_t* wb = wring + stage * C::kWStage;
           mbar_arrive_expect_tx(&wfull[stage], C::kTxW);
-          tma_load_2d(wb, &tm_w, &wfull[stage], kb * (kBlockK / 2), tile_n * kBlockN, pol_stream);
-          tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[stage], tile_n * kBlockN, kb * 2, pol_stream);
-          tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[stage], tile_n * kBlockN, kb * 2, pol_stream);
+          const int wr = wrow_of(tile_n);
+          tma_load_2d(wb, &tm_w, &wfull[stage], kb * (kBlockK / 2), wr, pol_stream);
+          tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[stage], wr, kb * 2, pol_stream);
+          tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[stage], wr, kb * 2, pol_stream);
           mbar_arrive_expect_tx(&xfull[stage], C::kTxX);
-          tma_load_2d(xring + stage * C::kXBytes, &tm_x, &xfull[stage], kb * kBlockK, tile_m * BT, pol_keep);
+          tma_load_2d(xring + stage * C::kXBytes, &tm_x, &xfull[stage], kb * kBlockK, xrow_of(tile_m), pol_keep);
         }
         issued |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | ((phase ^ 1u) << stage);
@@ -750,10 +800,11 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       }
       // scales of this tile, loaded before the accumulator is ready: s_c of this
       // thread's row, s_x of token m0 + lane of the first column chunk
-      const int n = tile_n * kBlockN + r;
-      const int m0 = tile_m * BT;
+      const int n = tile_n * kBlockN + r;  // output column (within the group)
+      const int m0 = xrow_of(tile_m);
+      const int mend = g_mend;             // rows from here on are not this tile's
       const bool n_ok = n < p.N;
-      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
+      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + g_scoff + n) : 0.0f;
       // the first token this warp writes: split-K clusters write only their own piece
       constexpr int SXC = CS >= 2 ? (C::kPieceT < 32 ? C::kPieceT : 32) : CH;
       const int sx0 = m0 + (CS >= 4 ? (int)(crank % C::kSlices) * C::kPieceT : 0);
@@ -761,9 +812,9 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       if constexpr (FQ) {
         // s_x from the quantizing warps (all four have arrived on xfirst)
         if (!__all_sync(0xffffffffu, mbar_wait(xfirst, 0, abort_flag))) goto epi_done;
-        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? sxs[sx0 - m0 + lane] : 0.0f;
+        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? sxs[sx0 - m0 + lane] : 0.0f;
       } else {
-        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < p.M) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
+        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
       }
       // split-K clusters: the scales of the piece this thread will write (the
       // reduce-scatter's owner phase), also loaded before the accumulator wait.
@@ -788,13 +839,13 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
       if constexpr (CS >= 2 && !OUT_I32) {
         if (onn_ok) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) osc[q4] = __ldg(p.s_c + onn + q4);
+          for (int q4 = 0; q4 < 4; ++q4) osc[q4] = __ldg(p.s_c + g_scoff + onn + q4);
         }
 #pragma unroll
         for (int j = 0; j < kSxRegs; ++j) {
           const int i = j * 32 + lane;
           const int m = m0 + ohh * C::kPieceT + ot0 + i * kWarpsPerPiece;
-          osl[j] = (i < kTok && m < p.M) ? (FQ ? sxs[m - m0] : __ldg(p.s_x + m)) : 0.0f;
+          osl[j] = (i < kTok && m < mend) ? (FQ ? sxs[m - m0] : __ldg(p.s_x + m)) : 0.0f;
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
@@ -891,7 +942,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
                 float sxm = 0.0f;
                 if constexpr (!OUT_I32)
                   sxm = __shfl_sync(0xffffffffu, (kSxRegs == 1 || (g0 + c) * 4 < 32) ? osl[0] : osl[kSxRegs - 1], i & 31);
-                if (i < kTok && m < p.M && onn_ok) {
+                if (i < kTok && m < mend && onn_ok) {
                   if constexpr (OUT_I32) {
                     *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.out) + (size_t)m * p.N + onn) = acc[c];
                   } else {
@@ -919,11 +970,11 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           for (int cc = 0; cc < BT / CH; ++cc) {
             const float sx_cur = sx_next;
             if (cc + 1 < BT / CH)
-              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < p.M) ? __ldg(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
+              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < mend) ? __ldg(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
             uint32_t v[32];
             tmem_load_cols<CH>(t_lane + cc * CH, v);
             if (whole) {
-              store_chunk<OUT_I32, CH>(p, m0 + cc * CH, n, n_ok, v, sx_cur, sc);
+              store_chunk<OUT_I32, CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
             } else {
 #pragma unroll
               for (int i = 0; i < CH; ++i) {
