@@ -430,8 +430,71 @@ def run_ours(args, rank, world, local_rank):
                            "frac_of_nominal_4500": g["gemm_tops"] / 4500.0,
                            "traffic": ncu_traffic("prefill")}
         res["prefill"] = pre
+        res["grouped"] = grouped_side(dev, int8_peak, hbm_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w)
+    return res
+
+
+def grouped_side(dev, int8_peak, hbm_peak, n=20):
+    """The grouped GEMM on a mixture-of-experts layer: 8 experts of the MLP up/gate
+    geometry (N=14336, K=4096), tokens routed top-2 by a seeded random assignment;
+    a decode batch (16 tokens -> 32 rows) and a prefill batch (4096 tokens -> 8192
+    rows).  n back-to-back grouped GEMMs in one CUDA graph between CUDA events.
+    The experts are one seeded expert quantized once and copied 8 times (separate
+    memory, so every expert's bytes are read from HBM; the values do not change
+    the timing)."""
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+    E, N, K = 8, 14336, 4096
+    w = synth.WORKLOADS["mlp_up"]
+    X, W = synth.make_workload(w)
+    qw, s_u8, a_u8, s_c = lq.lq_quantize_weights(W.to(dev))
+    qw_all = torch.cat([qw] * E)
+    s_all = torch.cat([s_u8] * E, dim=1).contiguous()
+    a_all = torch.cat([a_u8] * E, dim=1).contiguous()
+    sc_all = torch.cat([s_c] * E)
+    del qw, s_u8, a_u8, s_c
+    rng = np.random.default_rng(11)
+    stream = torch.cuda.Stream(dev)
+    res = {"workload": "mixture-of-experts up/gate layer: 8 experts N=14336 K=4096, top-2 routing",
+           "how": f"{n} back-to-back lq_w4a8_grouped_gemm calls in one CUDA graph between CUDA events"}
+    Xd = X.to(dev)
+    for name, tokens in (("decode", 16), ("prefill", 4096)):
+        rows = 2 * tokens
+        sizes = np.bincount(rng.integers(0, E, size=rows), minlength=E)
+        m_off = torch.from_numpy(np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)).to(dev)
+        src = Xd[torch.arange(rows, device=dev) % Xd.shape[0]]
+        xq, sx = lq.lq_quantize_act(src)
+        out = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                lq.lq_w4a8_grouped_gemm(xq, sx, qw_all, s_all, a_all, sc_all, m_off, N, out=out)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    lq.lq_w4a8_grouped_gemm(xq, sx, qw_all, s_all, a_all, sc_all, m_off, N, out=out)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            ts = []
+            for _ in range(3):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1) / n)
+        if lq.lq_get_device_error(dev) != 0:
+            raise RuntimeError("device error in the grouped measurement")
+        t_ms = sorted(ts)[1]
+        experts = int((sizes > 0).sum())
+        byts = experts * (N * K // 2 + 2 * N * K // 64 + 4 * N) + rows * K + 4 * rows + 2 * rows * N
+        ops = 2 * rows * N * K
+        gbs = byts / (t_ms * 1e-3) / 1e9
+        tops = ops / (t_ms * 1e-3) / 1e12
+        res[name] = {"rows": rows, "experts_used": experts, "us": 1e3 * t_ms, "gbs": gbs, "tops": tops,
+                     "frac_of_hbm": gbs / hbm_peak, "frac_of_int8": tops / int8_peak}
+        del xq, sx, out, src, g
     return res
 
 
