@@ -270,6 +270,34 @@ LQ_API lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const
                                       void* out_bf16, int M, int N, int K, int group, void* stream);
 
 /*
+ * lq_w4a8_gemm_ablation -- TEST AND MEASUREMENT ONLY: the pages' ablation of
+ * the dequantization arithmetic (LQQ) and of the pipeline (explicit
+ * coarse-grained, ExCP, vs implicit fine-grained, ImFP: LiquidGEMM Figs. 6
+ * and 13, as the review page's figure list and referee summary describe
+ * them), redone on sm_100 with four forms of the same tile kernel:
+ *   LQ_ABL_IMPLICIT (0): the product kernel -- SWAR expansion (one IMAD and
+ *     one XOR per four weights) into tensor memory, MMA with A from TMEM;
+ *   LQ_ABL_NAIVE (1): that pipeline with the weights expanded one at a time
+ *     (extract, IMAD, XOR, insert per weight);
+ *   LQ_ABL_EXPLICIT (2): SWAR expansion written to a shared-memory A tile
+ *     per slot (128-byte swizzle) and an MMA that reads both operands from
+ *     shared memory;
+ *   LQ_ABL_NAIVE_EXPLICIT (3): both.
+ *   Same operands, result and errors as lq_w4a8_gemm_ex with the tile
+ *   schedule; block_t must be 16 or 64 and split_k 4 (else
+ *   LQ_ERR_UNSUPPORTED_SHAPE); out_i32 as in lq_w4a8_gemm_ex.  Every variant
+ *   gives bit-identical results.
+ */
+#define LQ_ABL_IMPLICIT 0
+#define LQ_ABL_NAIVE 1
+#define LQ_ABL_EXPLICIT 2
+#define LQ_ABL_NAIVE_EXPLICIT 3
+LQ_API lq_status lq_w4a8_gemm_ablation(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                                       const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c, void* out,
+                                       int M, int N, int K, int group, int variant, int block_t, int split_k,
+                                       int out_i32, void* stream);
+
+/*
  * lq_w4a8_grouped_gemm -- the W4A8 GEMM for a mixture-of-experts layer (one
  * weight matrix per group, or expert, each applied to its own run of token
  * rows): out[m, n] = bf16((sum_k x_q[m,k] * Q_hat[e*N + n, k]) * s_x[m] *

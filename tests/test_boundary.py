@@ -159,3 +159,15 @@ def test_grouped_rejects_before_launch(lib):
     assert call(x=ODD) == 3 and call(out=ODD) == 3 and call(off=P((1 << 20) + 2)) == 3
     assert call(M=0) == 0                    # empty batch: nothing to launch
     assert call(M=-1) == 1
+
+
+def test_ablation_rejects_before_launch(lib):
+    f = lib.lq_w4a8_gemm_ablation
+
+    def call(variant=0, bt=16, split=4, M=16, N=256, K=512, x=GOOD, out=GOOD):
+        return f(x, GOOD, GOOD, GOOD, GOOD, GOOD, out, M, N, K, 64, variant, bt, split, 0, None)
+
+    assert call(variant=4) == 1 and call(variant=-1) == 1
+    assert call(bt=32) == 2 and call(bt=128) == 2 and call(split=2) == 2
+    assert call(K=192) == 2 and call(x=ODD) == 3 and call(out=P(0)) == 1
+    assert call(M=0) == 0

@@ -76,6 +76,7 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_linear_workspace_size_ex": ([I, I, I, I], Z),
             "lq_w4a8_linear_ex": ([P, P, P, P, P, P, I, I, I, I, P, Z, I, P], I),
             "lq_w4a8_grouped_gemm": ([P, P, P, P, P, P, P, I, P, I, I, I, I, P], I),
+            "lq_w4a8_gemm_ablation": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P], I),
             "lq_w4a8_grouped_gemm_ex": ([P, P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
@@ -329,6 +330,33 @@ def lq_w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N: int, out=None,
         _check("lq_w4a8_grouped_gemm", lib.lq_w4a8_grouped_gemm_ex(
             _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(m_off), G, _ptr(out),
             M, N, K, group, block_t, split_k, 1 if out_i32 else 0, _stream(x_q.device)))
+    return out
+
+
+# variants of lq_w4a8_gemm_ablation (LQ_ABL_* in lq.h)
+ABL_IMPLICIT, ABL_NAIVE, ABL_EXPLICIT, ABL_NAIVE_EXPLICIT = 0, 1, 2, 3
+
+
+def lq_w4a8_gemm_ablation(x_q, s_x, qw, s_u8, a_u8, s_c, variant: int, block_t: int, split_k: int = 4,
+                          out=None, group: int = GROUP, out_i32: bool = False):
+    """Test and measurement only: the GEMM with the dequantization arithmetic and pipeline
+    of one ablation variant (ABL_*), 16- or 64-token tiles in 4-CTA clusters."""
+    lib = load_library()
+    _need(x_q, torch.int8, "x_q")
+    M, K = x_q.shape
+    N = qw.shape[0]
+    _need(qw, torch.uint8, "qw", (N, K // 2))
+    if not out_i32:
+        _need(s_x, torch.float32, "s_x", (M,))
+        _need(s_c, torch.float32, "s_c", (N,))
+    odt = torch.int32 if out_i32 else torch.bfloat16
+    if out is None:
+        out = torch.empty(M, N, dtype=odt, device=x_q.device)
+    _need(out, odt, "out", (M, N))
+    with torch.cuda.device(x_q.device):
+        _check("lq_w4a8_gemm_ablation", lib.lq_w4a8_gemm_ablation(
+            _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out), M, N, K, group,
+            variant, block_t, split_k, 1 if out_i32 else 0, _stream(x_q.device)))
     return out
 
 

@@ -358,10 +358,39 @@ lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMa
   return LQ_ERR_INVALID_ARG;
 }
 
+// The ablation of the dequantization pipeline (GemmCfg's DQ): the same tile
+// kernel with per-element expansion (bit 0) and/or A expanded into shared
+// memory (bit 1), for 16- and 64-token tiles in 4-CTA clusters.
+template <int BT, int CS, bool I32, int DQ>
+lq_status launch_abl_t(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
+                       const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  using C = lq::GemmCfg<BT, CS, DQ>;
+  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32, false, DQ>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tw, ts, ta, a);
+}
+
+template <bool I32>
+lq_status launch_ablation(const Schedule& s, int dq, const CUtensorMap& tx, const CUtensorMap& tw,
+                          const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  if (dq == 0) return launch_gemm<I32>(s, tx, tw, ts, ta, a, st);
+  if (s.kind != kSchedTiles || s.cs != 4) return LQ_ERR_UNSUPPORTED_SHAPE;
+  switch (s.bt * 4 + dq) {
+    case 16 * 4 + 1: return launch_abl_t<16, 4, I32, 1>(s, tx, tw, ts, ta, a, st);
+    case 16 * 4 + 2: return launch_abl_t<16, 4, I32, 2>(s, tx, tw, ts, ta, a, st);
+    case 16 * 4 + 3: return launch_abl_t<16, 4, I32, 3>(s, tx, tw, ts, ta, a, st);
+    case 64 * 4 + 1: return launch_abl_t<64, 4, I32, 1>(s, tx, tw, ts, ta, a, st);
+    case 64 * 4 + 2: return launch_abl_t<64, 4, I32, 2>(s, tx, tw, ts, ta, a, st);
+    case 64 * 4 + 3: return launch_abl_t<64, 4, I32, 3>(s, tx, tw, ts, ta, a, st);
+  }
+  return LQ_ERR_UNSUPPORTED_SHAPE;
+}
+
 lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                     const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
                     void* workspace, size_t ws_bytes, int block_t, int schedule, int split_k, int grid,
-                    bool out_i32, void* stream) {
+                    bool out_i32, void* stream, int dq = 0) {
   lq_status st = check_gemm_shape(M, N, K, group);
   if (st != LQ_OK) return st;
   if (!valid_schedule(M, block_t, schedule, split_k, grid)) return LQ_ERR_INVALID_ARG;
@@ -411,6 +440,9 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   a.KB = s.KB;
   a.U = s.U;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (dq != 0)
+    return out_i32 ? launch_ablation<true>(s, dq, tx, tw, ts, ta, a, cs)
+                   : launch_ablation<false>(s, dq, tx, tw, ts, ta, a, cs);
   return out_i32 ? launch_gemm<true>(s, tx, tw, ts, ta, a, cs) : launch_gemm<false>(s, tx, tw, ts, ta, a, cs);
 }
 
@@ -614,6 +646,15 @@ lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* 
                            size_t workspace_bytes, void* stream) {
   return gemm_impl(x_q, nullptr, qw, s_u8, a_u8, nullptr, acc, M, N, K, group, workspace, workspace_bytes, 0,
                    0, 0, 0, true, stream);
+}
+
+lq_status lq_w4a8_gemm_ablation(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                                const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
+                                int variant, int block_t, int split_k, int out_i32, void* stream) {
+  if (variant < LQ_ABL_IMPLICIT || variant > LQ_ABL_NAIVE_EXPLICIT) return LQ_ERR_INVALID_ARG;
+  if ((block_t != 16 && block_t != 64) || split_k != 4) return LQ_ERR_UNSUPPORTED_SHAPE;
+  return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out, M, N, K, group, nullptr, 0, block_t, kSchedTiles, split_k,
+                   0, out_i32 != 0, stream, variant);
 }
 
 lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8, int N, int K,

@@ -360,4 +360,19 @@ __device__ __forceinline__ void lqq_expand_word(uint32_t w, uint32_t s, uint32_t
   hi = (((w >> 4) & 0x0F0F0F0Fu) * s + a4) ^ 0x80808080u;
 }
 
+// The same eight values one at a time (nibble extract, IMAD, XOR, byte insert
+// per weight): the per-element dequantization the SWAR form replaces, kept
+// for the ablation of the expansion arithmetic.  a is the plain u8 offset.
+__device__ __forceinline__ void naive_expand_word(uint32_t w, uint32_t s, uint32_t a, uint32_t& lo, uint32_t& hi) {
+  uint32_t r0 = 0u, r1 = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t q0 = (w >> (8 * i)) & 0xFu, q1 = (w >> (8 * i + 4)) & 0xFu;
+    r0 |= (((q0 * s + a) ^ 0x80u) & 0xFFu) << (8 * i);
+    r1 |= (((q1 * s + a) ^ 0x80u) & 0xFFu) << (8 * i);
+  }
+  lo = r0;
+  hi = r1;
+}
+
 }  // namespace lq

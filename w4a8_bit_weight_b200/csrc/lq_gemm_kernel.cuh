@@ -54,7 +54,12 @@ constexpr int kGemmThreads = 192;
 __host__ __device__ constexpr int round_up_c(int x, int a) { return (x + a - 1) / a * a; }
 __host__ __device__ constexpr int max_c(int a, int b) { return a > b ? a : b; }
 
-template <int BT, int CS>
+// DQ selects the expansion for the ablation of the dequantization pipeline
+// (the product path is DQ = 0): bit 0 = per-element expansion instead of the
+// SWAR form; bit 1 = the expanded weights go to a shared-memory A tile per
+// slot and the MMA reads both operands from shared memory (explicit
+// pipeline), instead of tensor memory (implicit pipeline).
+template <int BT, int CS, int DQ = 0>
 struct GemmCfg {
   static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128 || BT == 256, "tokens per tile");
   static_assert(CS >= 0 && CS <= 8, "cluster size");
@@ -84,19 +89,20 @@ struct GemmCfg {
   static constexpr int kPieceBytes = kPieceT * 32 * 4;            // [tokens][32 rows] int32
   static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * kOwned * kPieceBytes : 0;  // received pieces
   static constexpr int kXRing = kStages * kXBytes;
+  static constexpr int kASmem = (DQ & 2) ? kSlots * kBlockN * kBlockK : 0;  // explicit pipeline: int8 A tiles, SW128
   static constexpr int kWRing = kStages * kWStage;
   // mbarriers and flags in the first 512 bytes; with fused activation
   // quantization, the cluster's partial row maxima [CS][16] and s_x [16]
   // after; the expansion warps' progress counters [4] at byte 1088
   static constexpr int kBarBytes = 1152;
-  static constexpr int kUsed = kXRing + kWRing + kRedBytes + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kUsed = kXRing + kASmem + kWRing + kRedBytes + kBarBytes + 1024;  // + alignment slack
   // Shared memory also bounds how many CTAs share an SM: a 512-column CTA
   // takes at least 120 KB (one per SM), a 256-column CTA at least 80 KB (at
   // most two per SM), so co-resident CTAs never exceed the 512 TMEM columns.
   static constexpr int kSmemBytes = max_c(round_up_c(kUsed, 1024), kTmemCols == 512 ? 122880 : 81920);
   static_assert(kAccCols + kSlots * 32 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kXBytes % 1024 == 0 && (kXRing + kWRing + kRedBytes) % 8 == 0, "alignment");
+  static_assert(kXBytes % 1024 == 0 && (kXRing + kASmem + kWRing + kRedBytes) % 8 == 0, "alignment");
   static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 8 * 8 + 16 <= 512, "barrier area");
   // One K-block more than TMEM slots and no refills (a 16- or 32-token decode
   // CTA holding its whole K-slice): the extra block is expanded into the
@@ -250,13 +256,14 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&v)[32]
 // the expansion warps quantize them (per-token symmetric INT8, the same
 // arithmetic as quantize_act_kernel) straight into the swizzled activation
 // tiles; the row maxima are combined over the cluster through DSMEM.
-template <int BT, int CS, bool OUT_I32, bool FQ = false>
-__global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 256 ? 2 : 1)
+template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0>
+__global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols == 256 ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
                      const GemmArgs p) {
-  using C = GemmCfg<BT, CS>;
+  using C = GemmCfg<BT, CS, DQ>;
   static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
+  static_assert(DQ == 0 || (!FQ && CS >= 1), "ablation variants: plain tile schedules only");
   constexpr int S = C::kStages;
   constexpr int A = C::kSlots;
   // with as many TMEM slots as stages, block `it` uses stage and slot it % S:
@@ -266,9 +273,10 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xring = smem;                          // S x [BT][128] int8, SW128
-  uint8_t* wring = smem + C::kXRing;              // S x ([128][64] packed, SW64 | s [2][128] | a [2][128])
-  int32_t* red = reinterpret_cast<int32_t*>(smem + C::kXRing + C::kWRing);  // [CS-1][BT][128]
-  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::kXRing + C::kWRing + C::kRedBytes);
+  uint8_t* aring = smem + C::kXRing;              // explicit pipeline: A x [128][128] int8, SW128
+  uint8_t* wring = aring + C::kASmem;             // S x ([128][64] packed, SW64 | s [2][128] | a [2][128])
+  int32_t* red = reinterpret_cast<int32_t*>(wring + C::kWRing);  // [CS-1][BT][128]
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(wring + C::kWRing + C::kRedBytes);
   uint64_t* xfull = wfull + S;
   uint64_t* empty = xfull + S;
   uint64_t* afull = empty + S;    // [A]
@@ -397,7 +405,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
   }
 
   // the overflow K-block (see GemmCfg): one tile, exactly one block more than slots, no refills
-  const bool ovf = CS >= 1 && A >= 2 && (int)(u_end - u_begin) == A + 1 && A + 1 <= S;
+  const bool ovf = !(DQ & 2) && CS >= 1 && A >= 2 && (int)(u_end - u_begin) == A + 1 && A + 1 <= S;
 
   // Producer and MMA warps run their loops with all 32 lanes (one lane issues),
   // so every warp stays converged up to the CTA barrier at teardown.
@@ -541,10 +549,18 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           const int r_slot = min(run_ts, max(0, total - A - it));
           auto issue = [&](int r) {
             const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
-            const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
+            if constexpr ((DQ & 2) != 0) {
+              const uint64_t adesc = smem_desc_k_sw128(smem_u32(aring + slot * (kBlockN * kBlockK)));
 #pragma unroll
-            for (int j = 0; j < kBlockK / 32; ++j)
-              mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb + r > kb0 || j > 0) ? 1u : 0u);
+              for (int j = 0; j < kBlockK / 32; ++j)
+                mma_i8_ss(tmem_base, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
+                          (kb + r > kb0 || j > 0) ? 1u : 0u);
+            } else {
+              const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
+#pragma unroll
+              for (int j = 0; j < kBlockK / 32; ++j)
+                mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb + r > kb0 || j > 0) ? 1u : 0u);
+            }
           };
           int r = 0;
           for (; r < r_both; ++r) {
@@ -750,10 +766,17 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           const uint4 q = lds128(wrow + ((c ^ sw) << 4));
           const uint32_t s = c < 2 ? s0 : s1;
           const uint32_t a4 = c < 2 ? a0 : a1;
-          lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
-          lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
-          lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
-          lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
+          if constexpr ((DQ & 1) != 0) {
+            naive_expand_word(q.x, s, a4 & 0xFFu, v[8 * c + 0], v[8 * c + 1]);
+            naive_expand_word(q.y, s, a4 & 0xFFu, v[8 * c + 2], v[8 * c + 3]);
+            naive_expand_word(q.z, s, a4 & 0xFFu, v[8 * c + 4], v[8 * c + 5]);
+            naive_expand_word(q.w, s, a4 & 0xFFu, v[8 * c + 6], v[8 * c + 7]);
+          } else {
+            lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
+            lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
+            lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
+            lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
+          }
         }
         if (to_smem) {
           // row r of a 128-byte-swizzled K-major tile (the MMA's A descriptor)
@@ -765,8 +788,17 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS>::kTmemCols == 25
           __syncwarp();
           if (lane == 0) mbar_arrive(ovfull);
         } else {
-          tmem_st_32x32b_x32(t_lane + C::kAccCols + slot * 32, v);
-          tmem_st_wait();
+          if constexpr ((DQ & 2) != 0) {
+            // explicit pipeline: row r of the slot's 128-byte-swizzled A tile
+            uint8_t* orow = aring + slot * (kBlockN * kBlockK) + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(orow + ((c ^ (r & 7)) << 4)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            fence_proxy_async_smem();  // read by the tensor core through the async proxy
+          } else {
+            tmem_st_32x32b_x32(t_lane + C::kAccCols + slot * 32, v);
+            tmem_st_wait();
+          }
           tc_fence_before();
           // a refilled block's activation tile: one warp sees it land before
           // the slot is reported ready (the MMA warp waits for the slot only)
