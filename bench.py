@@ -431,6 +431,7 @@ def run_ours(args, rank, world, local_rank):
                            "traffic": ncu_traffic("prefill")}
         res["prefill"] = pre
         res["grouped"] = grouped_side(dev, int8_peak, hbm_peak)
+        res["ablation"] = ablation_side(dev, hbm_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w)
     return res
@@ -495,6 +496,64 @@ def grouped_side(dev, int8_peak, hbm_peak, n=20):
         res[name] = {"rows": rows, "experts_used": experts, "us": 1e3 * t_ms, "gbs": gbs, "tops": tops,
                      "frac_of_hbm": gbs / hbm_peak, "frac_of_int8": tops / int8_peak}
         del xq, sx, out, src, g
+    return res
+
+
+def ablation_side(dev, hbm_peak, n=40):
+    """The pages' ablation of the dequantization arithmetic and pipeline, redone on the
+    tile kernel: SWAR (LQQ) vs per-element expansion, A in tensor memory (implicit
+    pipeline) vs a shared-memory A tile (explicit pipeline).  A decode layer (16 tokens,
+    N = K = 4096, 16-token tiles) and a down-projection at 64 tokens (N = 4096,
+    K = 14336, 64-token tiles), both in 4-CTA clusters; n back-to-back launches per
+    variant in one CUDA graph, the weights rotating over L2-cold copies."""
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+    names = {lq.ABL_IMPLICIT: "lqq_implicit", lq.ABL_NAIVE: "naive_implicit", lq.ABL_EXPLICIT: "lqq_explicit",
+             lq.ABL_NAIVE_EXPLICIT: "naive_explicit"}
+    res = {"how": f"{n} back-to-back lq_w4a8_gemm_ablation calls per variant in one CUDA graph; us per launch",
+           "variants": "lqq = SWAR IMAD+XOR expansion, naive = one weight at a time; implicit = A in TMEM, "
+                       "explicit = A tile in shared memory"}
+    stream = torch.cuda.Stream(dev)
+    for label, (M, N, K, bt) in (("decode_16x4096x4096", (16, 4096, 4096, 16)),
+                                 ("down_64x4096x14336", (64, 4096, 14336, 64))):
+        X, W = synth.make_problem(M, N, K, seed=21, n_outliers=8)
+        qw, s_u8, a_u8, s_c = lq.lq_quantize_weights(W.to(dev))
+        wset = qw.numel() + 2 * s_u8.numel() + 4 * s_c.numel()
+        n_sets = min(48, max(4, int(np.ceil(3 * L2_BYTES / wset))))
+        sets = [(qw, s_u8, a_u8, s_c)] + [(qw.clone(), s_u8.clone(), a_u8.clone(), s_c.clone())
+                                          for _ in range(n_sets - 1)]
+        xq, sx = lq.lq_quantize_act(X.to(dev))
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        entry = {}
+        with torch.cuda.stream(stream):
+            for v, nm in names.items():
+                for i in range(2):
+                    lq.lq_w4a8_gemm_ablation(xq, sx, *sets[i % n_sets], v, bt, out=out)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(n):
+                        lq.lq_w4a8_gemm_ablation(xq, sx, *sets[i % n_sets], v, bt, out=out)
+                g.replay()
+                torch.cuda.synchronize(dev)
+                ts = []
+                for _ in range(3):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize(dev)
+                    ts.append(1e3 * e0.elapsed_time(e1) / n)
+                us = sorted(ts)[1]
+                gbs = gemm_bytes(M, N, K) / (us * 1e-6) / 1e9
+                entry[nm] = {"us": us, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
+                del g
+        if lq.lq_get_device_error(dev) != 0:
+            raise RuntimeError("device error in the ablation measurement")
+        base = entry["lqq_implicit"]["us"]
+        for nm in entry:
+            entry[nm]["slowdown_vs_lqq_implicit"] = entry[nm]["us"] / base
+        res[label] = entry
+        del sets, qw, s_u8, a_u8, s_c
     return res
 
 
