@@ -320,13 +320,15 @@ LQ_API lq_status lq_w4a8_gemm_ablation(const int8_t* x_q, const float* s_x, cons
  *   Requires N % 128 == 0 (a weight tile never spans two groups), the GEMM's
  *   K and group rules, 1 <= groups <= LQ_MAX_GROUPS, 16-byte-aligned
  *   x_q, qw, s_u8, a_u8, out and 4-byte-aligned s_x, s_c, m_off.  No
- *   workspace.  One thread-block cluster per 128-row weight tile and token
- *   tile (split-K inside the cluster for small token counts); clusters whose
- *   token tile lies past the last group's rows exit at once.
- * lq_w4a8_grouped_gemm_ex adds block_t (0 = from the mean rows per group,
- *   else 16, 32, 64 or 128), split_k (0 = automatic, else as in
- *   LQ_SCHED_TILES) and out_i32 (int32 accumulators to `out`, s_x and s_c
- *   unused).
+ *   workspace.  Groups of more than 128 rows on average (with N % 256 == 0
+ *   and K % 256 == 0) run on CTA pairs over 256 x 256 tiles; otherwise one
+ *   thread-block cluster per 128-row weight tile and token tile (split-K
+ *   inside the cluster for small token counts).  Tiles past the last group's
+ *   rows are skipped.
+ * lq_w4a8_grouped_gemm_ex adds block_t (0 = automatic, else 16, 32, 64 or 128
+ *   for the tile kernel, or 256 for CTA pairs, which need N % 256 == 0 and
+ *   K % 256 == 0), split_k (0 = automatic, else as in LQ_SCHED_TILES; none
+ *   with 256) and out_i32 (int32 accumulators to `out`, s_x and s_c unused).
  */
 #define LQ_MAX_GROUPS 1024
 LQ_API lq_status lq_w4a8_grouped_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw,

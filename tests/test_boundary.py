@@ -152,7 +152,8 @@ def test_grouped_rejects_before_launch(lib):
     assert call(N=192) == 2                  # a weight tile would span two groups
     assert call(N=200) == 2 and call(K=192) == 2 and call(group=32) == 2
     assert call(groups=0) == 1 and call(groups=lq.MAX_GROUPS + 1) == 1
-    assert call(bt=256) == 1 and call(bt=48) == 1 and call(split=-1) == 1
+    assert call(bt=48) == 1 and call(split=-1) == 1 and call(bt=256, split=2) == 1
+    assert call(bt=256, N=128) == 2 and call(bt=256, K=384) == 2   # pairs: N % 256, K % 256
     assert call(bt=64, split=8) == 1         # split 8 only for tiles of <= 32 tokens
     assert call(off=P(0)) == 1 and call(x=P(0)) == 1 and call(sc=P(0)) == 1
     assert call(i32=1, sc=P(0), sx=P(0)) != 1  # the int32 form takes no scales (then needs a device)

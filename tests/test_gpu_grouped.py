@@ -61,6 +61,9 @@ CASES = [
     ([130, 60], 256, 1024, 128, 4),
     ([0, 0, 5], 128, 256, 0, 0),                # leading empty groups
     ([1], 384, 512, 0, 0),                      # one group: the plain GEMM
+    ([300, 0, 520, 190], 256, 1024, 0, 0),      # > 128 rows per group: CTA pairs, ragged groups
+    ([3, 700, 40], 512, 512, 256, 0),           # CTA pairs forced, a small group among large ones
+    ([257], 256, 768, 256, 0),
 ]
 
 

@@ -778,32 +778,43 @@ lq_status grouped_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, c
   if (st != LQ_OK) return st;
   if (N % lq::kBlockN != 0) return LQ_ERR_UNSUPPORTED_SHAPE;  // a weight tile never spans two groups
   if (groups < 1 || groups > LQ_MAX_GROUPS || (long long)groups * N > INT_MAX) return LQ_ERR_INVALID_ARG;
-  if (block_t != 0 && (block_t == 256 || !valid_block_t(block_t))) return LQ_ERR_INVALID_ARG;
-  if (split_k < 0) return LQ_ERR_INVALID_ARG;
+  if (block_t != 0 && !valid_block_t(block_t)) return LQ_ERR_INVALID_ARG;
+  if (split_k < 0 || (block_t == 256 && split_k > 0)) return LQ_ERR_INVALID_ARG;
+  // 256-token tiles are the CTA-pair kernel's (256 weight rows, 256 K per stage)
+  if (block_t == 256 && (N % lq::kQBN != 0 || K % lq::kQBK != 0)) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return LQ_OK;
   if (!x_q || !qw || !s_u8 || !a_u8 || !out || !m_off || (!out_i32 && (!s_x || !s_c))) return LQ_ERR_INVALID_ARG;
   if (!aligned(x_q, 16) || !aligned(qw, 16) || !aligned(s_u8, 16) || !aligned(a_u8, 16) || !aligned(out, 16) ||
       !aligned(m_off, 4) || (s_x && !aligned(s_x, 4)) || (s_c && !aligned(s_c, 4)))
     return LQ_ERR_MISALIGNED;
-  // token tile from the mean rows per group; the token tiles of all groups
-  // number at most sum(ceil(M_e / bt)) <= (M + groups (bt - 1)) / bt, and at most M
-  const int bt = block_t ? block_t : auto_block_t((M + groups - 1) / groups);
+  // CTA pairs when the groups average more than 128 rows and the shape allows
+  // 256 x 256 tiles; else the tile kernel, its token tile from the mean rows
+  // per group.  The token tiles of all groups number at most
+  // sum(ceil(M_e / bt)) <= (M + groups (bt - 1)) / bt, and at most M.
+  const bool pair = block_t == 256 || (block_t == 0 && split_k == 0 && N % lq::kQBN == 0 &&
+                                       K % lq::kQBK == 0 && (long long)M > (long long)groups * lq::kPBT);
+  const int bt = pair ? lq::kQBT : block_t ? block_t : auto_block_t((M + groups - 1) / groups);
   if (split_k > 0 && !valid_split(bt, split_k)) return LQ_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
   const long long tm_bound = std::min<long long>(((long long)M + (long long)groups * (bt - 1)) / bt, M);
   if (tm_bound * bt > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
-  const Schedule s = make_schedule((int)(tm_bound * bt), N, K, bt, kSchedTiles, split_k, 0, dev->sms);
+  const Schedule s = pair ? make_schedule((int)(tm_bound * bt), N, K, 0, kSchedPair, 0, 0, dev->sms)
+                          : make_schedule((int)(tm_bound * bt), N, K, bt, kSchedTiles, split_k, 0, dev->sms);
   const int NT = groups * N;
+  // the pair kernel loads 128 tokens and 128 weight rows per CTA with 256 K per stage
+  const uint32_t x_rows = pair ? 128u : (uint32_t)bt;
+  const uint32_t w_box = pair ? (uint32_t)lq::kQBK / 2 : (uint32_t)lq::kBlockK / 2;
+  const uint32_t sa_groups = pair ? (uint32_t)lq::kQBK / LQ_GROUP : 2u;
   CUtensorMap tx, tw, ts, ta;
-  if (!make_map_u8(&tx, x_q, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, (uint32_t)bt,
+  if (!make_map_u8(&tx, x_q, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, x_rows,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)NT, (uint64_t)K / 2, lq::kBlockK / 2, lq::kBlockN,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_u8(&ts, s_u8, (uint64_t)NT, (uint64_t)K / LQ_GROUP, (uint64_t)NT, lq::kBlockN, 2u,
+      !make_map_u8(&tw, qw, (uint64_t)K / 2, (uint64_t)NT, (uint64_t)K / 2, w_box, lq::kBlockN,
+                   pair ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_u8(&ts, s_u8, (uint64_t)NT, (uint64_t)K / LQ_GROUP, (uint64_t)NT, lq::kBlockN, sa_groups,
                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_u8(&ta, a_u8, (uint64_t)NT, (uint64_t)K / LQ_GROUP, (uint64_t)NT, lq::kBlockN, 2u,
+      !make_map_u8(&ta, a_u8, (uint64_t)NT, (uint64_t)K / LQ_GROUP, (uint64_t)NT, lq::kBlockN, sa_groups,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return LQ_ERR_CUDA;
   lq::GemmArgs a;

@@ -154,6 +154,43 @@ __device__ __forceinline__ long long cta_of_unit(long long u, long long U, long 
   return ((u + 1) * G + U - 1) / U - 1;
 }
 
+// Grouped GEMM: the group of token tile j, the token tiles of all groups
+// numbered in group order (ceil(rows / bt) tiles per group).  Called by a
+// whole warp: each lane takes one group per step, an inclusive prefix sum of
+// the tile counts (shuffles) and a ballot find the group.  Returns the group,
+// or -1 past the last group's rows, and the tile's first row and the group's
+// end row.  Offsets are read clamped to [0, M]: whatever they hold, no row
+// outside the activations and the output is ever addressed.
+__device__ __forceinline__ int find_group_tile(const int* m_off, int groups, int M, int bt, int j, int& row0,
+                                               int& mend) {
+  const int lane = threadIdx.x & 31;
+  auto off_at = [&](int e) { return min(max(__ldg(m_off + e), 0), M); };
+  int ge = -1, before = 0, run = 0;
+  for (int base = 0; base < groups && ge < 0; base += 32) {
+    const int e = base + lane;
+    int cnt = 0;
+    if (e < groups) cnt = max(0, off_at(e + 1) - off_at(e) + bt - 1) / bt;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && j >= run + incl - cnt && j < run + incl);
+    if (hit) {
+      const int l = __ffs(hit) - 1;
+      ge = base + l;
+      before = run + __shfl_sync(0xffffffffu, incl - cnt, l);
+    }
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (ge >= 0) {
+    row0 = off_at(ge) + (j - before) * bt;
+    mend = off_at(ge + 1);
+  }
+  return ge;
+}
+
 // One lane polls the barrier; the decision is broadcast to the warp (cheaper
 // than 32 lanes polling the same mbarrier).
 __device__ __forceinline__ bool lane0_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -303,38 +340,15 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   // Grouped GEMM: this cluster's tile (token tile j over all groups, weight
   // tile tn of its group).  The row offsets may come from the preceding
   // kernel, so the dependency wait comes first.  Every warp finds the group
-  // itself (a scan of the groups' tile counts); a tile past the last group's
-  // rows leaves at once, before any barrier, in every CTA of its cluster.
+  // itself; a tile past the last group's rows leaves at once, before any
+  // barrier, in every CTA of its cluster.
   int g_xrow = 0, g_mend = p.M, g_wrow = 0, g_scoff = 0;
   if (p.m_off != nullptr) {
     griddep_wait();
     const int t = (int)(blockIdx.x / (CS >= 1 ? CS : 1));
     const int j = t % p.tiles_m, tn = t / p.tiles_m;
-    // offsets are read clamped to [0, M]: whatever they hold, no row outside
-    // the activations and the output is ever written
-    auto off_at = [&](int e) { return min(max(__ldg(p.m_off + e), 0), p.M); };
-    int ge = -1, before = 0, run = 0;
-    for (int base = 0; base < p.groups && ge < 0; base += 32) {
-      const int e = base + lane;
-      int cnt = 0;
-      if (e < p.groups) cnt = max(0, off_at(e + 1) - off_at(e) + BT - 1) / BT;
-      int incl = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && j >= run + incl - cnt && j < run + incl);
-      if (hit) {
-        const int l = __ffs(hit) - 1;
-        ge = base + l;
-        before = run + __shfl_sync(0xffffffffu, incl - cnt, l);
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
+    const int ge = find_group_tile(p.m_off, p.groups, p.M, BT, j, g_xrow, g_mend);
     if (ge < 0) return;
-    g_xrow = off_at(ge) + (j - before) * BT;
-    g_mend = off_at(ge + 1);
     g_wrow = ge * p.N + tn * kBlockN;
     g_scoff = ge * p.N;
   }

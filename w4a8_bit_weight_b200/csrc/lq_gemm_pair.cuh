@@ -117,9 +117,9 @@ __device__ __forceinline__ uint32_t idesc_i8_pair(int n) {
 // half per pair, so that round takes half as long.
 struct PairWork {
   int nwhole, nunits, tail_tile, tail_half;
-  __device__ __forceinline__ PairWork(int cid, int ncl, int tiles) {
+  __device__ __forceinline__ PairWork(int cid, int ncl, int tiles, bool may_split) {
     const int rounds = tiles / ncl, rem = tiles - rounds * ncl;
-    const bool split = rem > 0 && 2 * rem <= ncl;
+    const bool split = may_split && rem > 0 && 2 * rem <= ncl;
     nwhole = split ? rounds : (cid < tiles ? (tiles - 1 - cid) / ncl + 1 : 0);
     nunits = nwhole + ((split && cid < 2 * rem) ? 1 : 0);
     tail_tile = rounds * ncl + (cid >> 1);
@@ -219,19 +219,54 @@ __global__ void __launch_bounds__(kQThreads, 1)
   const int tiles = (int)(p.U);             // host passes the tile count in U
   const int cid = blockIdx.x >> 1;
   const int ncl = gridDim.x >> 1;
-  const PairWork pw(cid, ncl, tiles);
-  const int total = pw.nunits * KS;         // K-blocks this CTA takes part in
+  // Grouped GEMM (m_off set): the tiles are the token tiles of all groups (a
+  // bound) times the weight tiles of one group; every role finds a tile's
+  // group from the offsets (read after the grid dependency wait) and skips
+  // tiles past the last group's rows, so all roles step through the same
+  // tiles.  The last round is not split in token halves then.
+  const bool grouped = (p.m_off != nullptr);
+  const PairWork pw(cid, ncl, tiles, !grouped);
+  // first token row, end row, first (stacked) weight row and scale offset of a
+  // tile; false: no rows (grouped only).  Called by whole warps.
+  auto geo = [&](int tile, int& xrow0, int& mend, int& wrow0, int& scoff) -> bool {
+    const int tm = tile % tiles_m, tn = tile / tiles_m;
+    if (!grouped) {
+      xrow0 = tm * kQBT;
+      mend = p.M;
+      wrow0 = tn * kQBN;
+      scoff = 0;
+      return true;
+    }
+    const int ge = find_group_tile(p.m_off, p.groups, p.M, kQBT, tm, xrow0, mend);
+    if (ge < 0) return false;
+    wrow0 = ge * p.N + tn * kQBN;
+    scoff = ge * p.N;
+    return true;
+  };
+  int nvalid = pw.nunits;
+  if (grouped && warp >= 2 && warp < kQEpiWarp0) {
+    griddep_wait();
+    nvalid = 0;
+    for (int k = 0; k < pw.nunits; ++k) {
+      int a0, a1, a2, a3;
+      if (geo(pw.tile(k, cid, ncl), a0, a1, a2, a3)) ++nvalid;
+    }
+  }
+  const int total = nvalid * KS;            // K-blocks this CTA takes part in
 
   if (warp == 0) {
     // ---------------------------------------------------- weight producer
     // weights depend on nothing the preceding kernel writes: no dependency wait
     uint64_t pol = 0;
     if (leader) pol = l2_policy_evict_first();
+    if (grouped) griddep_wait();  // which weights: from the offsets
     uint32_t issued = 0, issued_par = 0;
     int it = 0;
     for (int k = 0; k < pw.nunits; ++k) {
       const int tile = pw.tile(k, cid, ncl);
-      const int wrow = (tile / tiles_m) * kQBN + (int)crank * 128;
+      int xr0, me, wr0, so;
+      if (!geo(tile, xr0, me, wr0, so)) continue;
+      const int wrow = wr0 + (int)crank * 128;
       for (int kb = 0; kb < KS; ++kb, ++it) {
         const int w = it % SW;
         const uint32_t use = (uint32_t)(it / SW);
@@ -265,9 +300,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
     int it = 0;
     for (int k = 0; k < pw.nunits; ++k) {
       const int tile = pw.tile(k, cid, ncl), half = pw.half(k);
+      int xr0, me, wr0, so;
+      if (!geo(tile, xr0, me, wr0, so)) continue;
       // B is split by N across the pair: 128 tokens per CTA, 64 for a half tile
       // (the 128-row box then carries 64 rows the MMA does not read)
-      const int xrow = (tile % tiles_m) * kQBT + (half < 0 ? (int)crank * 128 : half * 128 + (int)crank * 64);
+      const int xrow = xr0 + (half < 0 ? (int)crank * 128 : half * 128 + (int)crank * 64);
       for (int kb = 0; kb < KS; ++kb, ++it) {
         const int x = it % SX;
         const uint32_t use = (uint32_t)(it / SX);
@@ -296,7 +333,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
       // ------------------------------------------------- MMA issuer (even CTA)
       bool any = false;
       int it = 0, j = 0;
-      for (int k = 0; k < pw.nunits; ++k, ++j) {
+      if (grouped) griddep_wait();
+      for (int k = 0; k < pw.nunits; ++k) {
+        if (grouped) {
+          int a0, a1, a2, a3;
+          if (!geo(pw.tile(k, cid, ncl), a0, a1, a2, a3)) continue;
+        }
         const uint32_t idesc = idesc_i8_pair(pw.half(k) < 0 ? kQBT : kQBT / 2);
         // the single accumulator is free once both CTAs' epilogues have loaded it
         if (!warp_wait(accempty, ((uint32_t)j & 1u) ^ 1u, abort_flag, true)) goto mma_done;
@@ -319,6 +361,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
         if (leader) tc_commit_pair_mc(accfull, 0x3);
         __syncwarp();
+        ++j;
       }
       griddep_launch_dependents();
     mma_done:
@@ -383,16 +426,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     griddep_wait();
     int j = 0;
-    for (int k = 0; k < pw.nunits; ++k, ++j) {
+    for (int k = 0; k < pw.nunits; ++k) {
       const int tile = pw.tile(k, cid, ncl), half = pw.half(k);
-      const int tm = tile % tiles_m, tn = tile / tiles_m;
-      const int n = tn * kQBN + (int)crank * 128 + r;
+      int xr0, mend, wr0, scoff;
+      if (!geo(tile, xr0, mend, wr0, scoff)) continue;
+      const int tn = tile / tiles_m;
+      const int n = tn * kQBN + (int)crank * 128 + r;  // output column (within the group)
       const bool n_ok = n < p.N;
       // a half tile's 128 tokens are accumulator columns 0-127: the second
       // pair of warps only hands the accumulator back
-      const int mb = tm * kQBT + (half < 0 ? e * 128 : half * 128);
+      const int mb = xr0 + (half < 0 ? e * 128 : half * 128);
+      const int jj = j++;
       if (half >= 0 && e == 1) {
-        if (!warp_wait(accfull, (uint32_t)j & 1u, abort_flag, false)) goto epi_done;
+        if (!warp_wait(accfull, (uint32_t)jj & 1u, abort_flag, false)) goto epi_done;
         tc_fence_after();
         tc_fence_before();
         __syncwarp();
@@ -400,14 +446,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
         continue;
       }
       // scales are loaded before the accumulator is ready, off the hand-back path
-      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + n) : 0.0f;
+      const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + scoff + n) : 0.0f;
       float sx4[4];  // s_x of tokens mb + 32c + lane
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int m = mb + 32 * c + lane;
-        sx4[c] = (!OUT_I32 && m < p.M) ? __ldg(p.s_x + m) : 0.0f;
+        sx4[c] = (!OUT_I32 && m < mend) ? __ldg(p.s_x + m) : 0.0f;
       }
-      if (!warp_wait(accfull, (uint32_t)j & 1u, abort_flag, false)) goto epi_done;
+      if (!warp_wait(accfull, (uint32_t)jj & 1u, abort_flag, false)) goto epi_done;
       tc_fence_after();
       if constexpr (OUT_I32) {
 #pragma unroll 1
@@ -423,7 +469,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int m = mb + cc * 32 + i;
-            if (m < p.M && n_ok) reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)v[i];
+            if (m < mend && n_ok) reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)v[i];
           }
         }
       } else {
@@ -464,7 +510,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
           const uint32_t lo = odd ? (other >> 16) : (mine & 0xFFFFu);
           const uint32_t hi = odd ? (mine >> 16) : (other & 0xFFFFu);
           const int m = mb + 2 * q + (odd ? 1 : 0);
-          if (m < p.M && n0_ok)
+          if (m < mend && n0_ok)
             *reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.N + n0) =
                 lo | (hi << 16);
         }
