@@ -341,6 +341,17 @@ LQ_API lq_status lq_w4a8_grouped_gemm_ex(const int8_t* x_q, const float* s_x, co
                                          int group, int block_t, int split_k, int out_i32, void* stream);
 
 /*
+ * lq_test_wait_timeout -- TEST ONLY: launches a one-CTA kernel whose first
+ * warp waits on an mbarrier that nothing completes, with the GEMM kernels'
+ * bounded wait: after the 2 s limit it raises the CTA's abort flag and
+ * records LQ_ERR_TIMEOUT in the device error word; a second warp waiting on
+ * another such barrier leaves as soon as the flag is up.  No fault, no trap:
+ * the context stays usable, and lq_get_device_error then returns
+ * LQ_ERR_TIMEOUT once.
+ */
+LQ_API lq_status lq_test_wait_timeout(void* stream);
+
+/*
  * lq_get_device_error -- synchronizes `stream`, then reads and clears the
  * library's device error word.  Returns LQ_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last call (its output is then undefined),

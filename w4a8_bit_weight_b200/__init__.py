@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_linear_ex": ([P, P, P, P, P, P, I, I, I, I, P, Z, I, P], I),
             "lq_w4a8_grouped_gemm": ([P, P, P, P, P, P, P, I, P, I, I, I, I, P], I),
             "lq_w4a8_gemm_ablation": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P], I),
+            "lq_test_wait_timeout": ([P], I),
             "lq_w4a8_grouped_gemm_ex": ([P, P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
@@ -373,6 +374,14 @@ def lq_dequant_weights_i8(qw, s_u8, a_u8, group: int = GROUP, out=None):
         _check("lq_dequant_weights_i8", lib.lq_dequant_weights_i8(
             _ptr(qw), _ptr(s_u8), _ptr(a_u8), N, K, group, _ptr(out), _stream(qw.device)))
     return out
+
+
+def lq_test_wait_timeout(device=None) -> None:
+    """Test only: a kernel whose bounded waits run out (about 2 s); see lq.h."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check("lq_test_wait_timeout", lib.lq_test_wait_timeout(_stream(dev)))
 
 
 def lq_get_device_error(device=None) -> int:

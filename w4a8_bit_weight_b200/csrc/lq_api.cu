@@ -675,6 +675,14 @@ lq_status lq_dequant_weights_i8(const uint8_t* qw, const uint8_t* s_u8, const ui
   return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
 }
 
+lq_status lq_test_wait_timeout(void* stream) {
+  DeviceInfo* dev = nullptr;
+  const lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  lq::wait_timeout_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
 lq_status lq_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LQ_ERR_CUDA;
   unsigned int code = 0;

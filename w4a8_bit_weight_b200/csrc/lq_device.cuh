@@ -81,6 +81,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Test of the bounded waits (no fault, no trap): warp 0 waits on a barrier
+// that nothing completes and gives up after kWaitLimitNs, raising the CTA
+// abort flag and recording kErrTimeout; warp 1 waits on another such barrier
+// and must leave as soon as the flag is up, not after its own limit.
+__global__ void wait_timeout_kernel() {
+  __shared__ uint64_t bar[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) mbar_wait(&bar[threadIdx.x >> 5], 0, &abort_flag);
+  __syncthreads();
+}
+
 // Cluster-scope wait: also makes visible the shared-memory writes that other
 // CTAs of the cluster released before arriving (remote arrive with .release).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
