@@ -17,13 +17,22 @@
 //              one XOR per four weights) into the TMEM A slot of the stage,
 //              then the epilogue: int32 accumulators -> scales -> bf16.
 //
+// Hand-offs: the weights of a K-block complete on its stage's weight barrier,
+// the preloaded activation tiles on one barrier, a refilled activation tile
+// on its stage's barrier (waited for by one expansion warp before its slot is
+// reported ready).  The expansion warps publish how many blocks they have
+// handed over; the MMA thread issues every block known to be ready as one
+// run.  Stages and slots go back to the producer through MMA commits.
+//
 // Schedules (CS template parameter):
 //   CS >= 1  split-K inside a thread-block cluster of CS CTAs: the cluster
 //            owns one 128-row x BT-token tile, CTA rank r takes the r-th
-//            slice of the K-blocks.  The non-leader CTAs write their int32
-//            partial sums into the leader's shared memory (DSMEM) and arrive
-//            on its mbarrier; the leader adds them and runs the epilogue.
-//            CS = 1 is the plain one-CTA-per-tile schedule.
+//            slice of the K-blocks.  The partial sums are reduce-scattered
+//            through distributed shared memory: each CTA owns one piece of
+//            the tile (row quarters, token halves of them when CS = 8),
+//            receives the other CTAs' partials of it by bulk copies, adds
+//            them and writes that piece of the output.  CS = 1 is the plain
+//            one-CTA-per-tile schedule.
 //   CS == 0  stream-K over any grid: the M x N x K work is cut into units of
 //            one tile x one K-block of 128; CTA c takes units
 //            [c*U/G, (c+1)*U/G).  Tiles shared by several CTAs are summed in
@@ -38,6 +47,11 @@
 // stages before griddepcontrol.wait (weights are never written by the kernel
 // this launch overlaps), and the activation loads after it; the epilogue
 // waits before it reads scales or writes the output.
+//
+// Also here: the grouped form (GemmArgs::m_off, one weight matrix per group
+// of token rows, each cluster finding its group on the device), the fused
+// activation quantization (FQ) and the variants of the dequantization
+// ablation (DQ).
 #pragma once
 
 #include <cuda_bf16.h>
