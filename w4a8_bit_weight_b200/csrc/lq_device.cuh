@@ -63,6 +63,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Loads of data that the preceding kernel may write (activations, their
+// scales, group row offsets), made after griddepcontrol.wait.  Under
+// programmatic dependent launch that kernel is still running while this one
+// is resident, so the non-coherent read-only path (whose data must not change
+// during the kernel's lifetime) is not used for them: they are read through
+// L2 (ld.global.cg).
+template <typename T>
+__device__ __forceinline__ T ld_dep(const T* ptr) {
+  return __ldcg(ptr);
+}
+
 // Waits for the phase with the given parity to complete.  Gives up when the
 // CTA-wide abort flag is raised by another role, or after kWaitLimitNs (then
 // it raises the flag itself and records the error).  Returns false on give-up.

@@ -178,7 +178,7 @@ __device__ __forceinline__ long long cta_of_unit(long long u, long long U, long 
 __device__ __forceinline__ int find_group_tile(const int* m_off, int groups, int M, int bt, int j, int& row0,
                                                int& mend) {
   const int lane = threadIdx.x & 31;
-  auto off_at = [&](int e) { return min(max(__ldg(m_off + e), 0), M); };
+  auto off_at = [&](int e) { return min(max(ld_dep(m_off + e), 0), M); };
   int ge = -1, before = 0, run = 0;
   for (int base = 0; base < groups && ge < 0; base += 32) {
     const int e = base + lane;
@@ -278,7 +278,7 @@ __device__ __forceinline__ void store_out(const GemmArgs& p, int m, int n, int32
   if constexpr (OUT_I32) {
     reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = acc;
   } else {
-    const float scale = __fmul_rn(__ldg(p.s_x + m), sc);
+    const float scale = __fmul_rn(ld_dep(p.s_x + m), sc);
     const float y = __fmul_rn(__int2float_rn(acc), scale);
     reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
   }
@@ -678,7 +678,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
         const bool ld = has && m < p.M;
         const uint4* src = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)(ld ? m : 0) * p.K + (ld ? k0 : 0));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) xv[i][c] = ld ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < 4; ++c) xv[i][c] = ld ? ld_dep(src + c) : make_uint4(0u, 0u, 0u, 0u);
       }
       float pm[4];
 #pragma unroll
@@ -874,7 +874,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
         if (!__all_sync(0xffffffffu, mbar_wait(xfirst, 0, abort_flag))) goto epi_done;
         sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? sxs[sx0 - m0 + lane] : 0.0f;
       } else {
-        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? __ldg(p.s_x + sx0 + lane) : 0.0f;
+        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? ld_dep(p.s_x + sx0 + lane) : 0.0f;
       }
       // split-K clusters: the scales of the piece this thread will write (the
       // reduce-scatter's owner phase), also loaded before the accumulator wait.
@@ -905,7 +905,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
         for (int j = 0; j < kSxRegs; ++j) {
           const int i = j * 32 + lane;
           const int m = m0 + ohh * C::kPieceT + ot0 + i * kWarpsPerPiece;
-          osl[j] = (i < kTok && m < mend) ? (FQ ? sxs[m - m0] : __ldg(p.s_x + m)) : 0.0f;
+          osl[j] = (i < kTok && m < mend) ? (FQ ? sxs[m - m0] : ld_dep(p.s_x + m)) : 0.0f;
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
@@ -1030,7 +1030,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
           for (int cc = 0; cc < BT / CH; ++cc) {
             const float sx_cur = sx_next;
             if (cc + 1 < BT / CH)
-              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < mend) ? __ldg(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
+              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < mend) ? ld_dep(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
             uint32_t v[32];
             tmem_load_cols<CH>(t_lane + cc * CH, v);
             if (whole) {

@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int m = mb + 32 * c + lane;
-        sx4[c] = (!OUT_I32 && m < mend) ? __ldg(p.s_x + m) : 0.0f;
+        sx4[c] = (!OUT_I32 && m < mend) ? ld_dep(p.s_x + m) : 0.0f;
       }
       if (!warp_wait(accfull, (uint32_t)jj & 1u, abort_flag, false)) goto epi_done;
       tc_fence_after();

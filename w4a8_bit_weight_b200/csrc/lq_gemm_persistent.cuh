@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         const int mb = m0 + cc * 32;
         float sxl = 0.0f;
-        if (!OUT_I32 && mb + lane < p.M) sxl = __ldg(p.s_x + mb + lane);
+        if (!OUT_I32 && mb + lane < p.M) sxl = ld_dep(p.s_x + mb + lane);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int m = mb + i;

@@ -134,28 +134,47 @@ __global__ void __launch_bounds__(kQuantActThreads) quantize_act_kernel(const ui
   griddep_wait();               // X may be the output of the preceding kernel
   const int m = blockIdx.x;
   const uint16_t* row = X + (size_t)m * K;
-  float amax = 0.0f;
-  for (int k = threadIdx.x * 8; k < K; k += kQuantActThreads * 8) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + k));
+  // The first kActHold chunks of 8 values per thread (K <= 16384) stay in
+  // registers between the two passes; longer rows read the rest twice.
+  constexpr int kActHold = 8;
+  constexpr int kStep = kQuantActThreads * 8;
+  auto row_max = [](const uint4& v, float a) {
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w4[i] & 0xFFFFu)));
-      amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w4[i] >> 16)));
+      a = fmaxf(a, fabsf(bf16_bits_to_f32(w4[i] & 0xFFFFu)));
+      a = fmaxf(a, fabsf(bf16_bits_to_f32(w4[i] >> 16)));
     }
+    return a;
+  };
+  uint4 hold[kActHold];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kActHold; ++i) {
+    const int k = threadIdx.x * 8 + i * kStep;
+    hold[i] = k < K ? ld_dep(reinterpret_cast<const uint4*>(row + k)) : make_uint4(0u, 0u, 0u, 0u);
+    amax = row_max(hold[i], amax);
   }
+  for (int k = threadIdx.x * 8 + kActHold * kStep; k < K; k += kStep)
+    amax = row_max(ld_dep(reinterpret_cast<const uint4*>(row + k)), amax);
   amax = block_max<kQuantActThreads>(amax, red);
   const bool zero = (amax == 0.0f);
   const float inv = zero ? 0.0f : __fdiv_rn(127.0f, amax);
   if (threadIdx.x == 0) s_x[m] = zero ? 1.0f : __fdiv_rn(amax, 127.0f);
   int8_t* out = x_q + (size_t)m * K;
-  for (int k = threadIdx.x * 8; k < K; k += kQuantActThreads * 8) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + k));
+  auto quant8 = [&](const uint4& v, int k) {
     uint2 o;
     o.x = quant_pair_i8(v.x, inv) | (quant_pair_i8(v.y, inv) << 16);
     o.y = quant_pair_i8(v.z, inv) | (quant_pair_i8(v.w, inv) << 16);
     *reinterpret_cast<uint2*>(out + k) = o;
+  };
+#pragma unroll
+  for (int i = 0; i < kActHold; ++i) {
+    const int k = threadIdx.x * 8 + i * kStep;
+    if (k < K) quant8(hold[i], k);
   }
+  for (int k = threadIdx.x * 8 + kActHold * kStep; k < K; k += kStep)
+    quant8(ld_dep(reinterpret_cast<const uint4*>(row + k)), k);
 }
 
 // ---------------------------------------------------------------------------
