@@ -79,6 +79,9 @@ def _load():
         "lq_oracle_epilogue": [P, P, P, I, I, P],
         "lq_oracle_w4a8_gemm": [P, P, P, P, P, P, I, I, I, I, P, P],
         "lq_oracle_w4a8_gemm_sampled": [P, P, P, P, P, P, I, I, I, I, P, P, ctypes.c_int64, P, P],
+        "lq_oracle_quantize_weights_w4": [P, I, I, P, P],
+        "lq_oracle_quantize_act_f8": [P, I, I, P, P],
+        "lq_oracle_w4f8_gemm": [P, ctypes.c_float, P, P, I, I, I, P, P],
     }.items():
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -87,6 +90,10 @@ def _load():
     lib.lq_oracle_f32_to_bf16.restype = ctypes.c_uint16
     lib.lq_oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
     lib.lq_oracle_bf16_to_f32.restype = ctypes.c_float
+    lib.lq_oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    lib.lq_oracle_e4m3_to_f32.restype = ctypes.c_float
+    lib.lq_oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+    lib.lq_oracle_f32_to_e4m3.restype = ctypes.c_uint8
     lib.lq_oracle_num_threads.argtypes = []
     lib.lq_oracle_num_threads.restype = I
     _lib = lib
@@ -257,4 +264,56 @@ def w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N: int, group: int =
                          np.asarray(s_c)[e * N:(e + 1) * N], group)
         out[r0:r1] = o
         acc[r0:r1] = a
+    return out, acc
+
+
+# ---------------------------------------------------------------------------
+# W4 x FP8 variant (FireQ page, abstract): per-channel symmetric INT4 weights,
+# FP8 e4m3 activations with one scale per tensor.  Readings in lq_oracle.c.
+# ---------------------------------------------------------------------------
+
+def e4m3_to_f32(code: int) -> float:
+    """Value of an e4m3 code (1-4-3, bias 7, subnormals, NaN = S.1111.111)."""
+    return float(_load().lq_oracle_e4m3_to_f32(int(code) & 0xFF))
+
+
+def f32_to_e4m3(x: float) -> int:
+    """e4m3 code of a float: round to nearest even, finite values beyond 448 saturated."""
+    return int(_load().lq_oracle_f32_to_e4m3(float(x)))
+
+
+def quantize_weights_w4(W: np.ndarray):
+    """Per-channel symmetric INT4 in [-7, 7], stored as q + 8 in the LiquidQuant nibble layout.
+    W: uint16 [N,K] (bf16 bits).  Returns (qw4 [N,K/2] uint8, s_w [N] float32)."""
+    W = np.ascontiguousarray(W, np.uint16)
+    N, K = W.shape
+    qw4 = np.empty((N, K // 2), np.uint8)
+    s_w = np.empty(N, np.float32)
+    _check(_load().lq_oracle_quantize_weights_w4(_p(W), N, K, _p(qw4), _p(s_w)), "quantize_weights_w4")
+    return qw4, s_w
+
+
+def quantize_act_f8(X: np.ndarray):
+    """FP8 e4m3 codes of X * (448 / amax(X)) with one scale s_x = amax / 448 for the tensor.
+    X: uint16 [M,K] (bf16 bits).  Returns (x_f8 [M,K] uint8, s_x float32 scalar)."""
+    X = np.ascontiguousarray(X, np.uint16)
+    M, K = X.shape
+    x_f8 = np.empty((M, K), np.uint8)
+    s_x = np.empty(1, np.float32)
+    _check(_load().lq_oracle_quantize_act_f8(_p(X), M, K, _p(x_f8), _p(s_x)), "quantize_act_f8")
+    return x_f8, np.float32(s_x[0])
+
+
+def w4f8_gemm(x_f8, s_x, qw4, s_w):
+    """acc[m,n] = sum_k e4m3(x)[m,k] * (u[n,k] - 8), exact (float64); out = bf16(float(acc) * (s_x * s_w[n])).
+    Returns (out uint16 [M,N], acc float64 [M,N])."""
+    x_f8 = np.ascontiguousarray(x_f8, np.uint8)
+    qw4 = np.ascontiguousarray(qw4, np.uint8)
+    s_w = np.ascontiguousarray(s_w, np.float32)
+    M, K = x_f8.shape
+    N = qw4.shape[0]
+    out = np.empty((M, N), np.uint16)
+    acc = np.empty((M, N), np.float64)
+    _check(_load().lq_oracle_w4f8_gemm(_p(x_f8), float(s_x), _p(qw4), _p(s_w), M, N, K, _p(out), _p(acc)),
+           "w4f8_gemm")
     return out, acc

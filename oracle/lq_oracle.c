@@ -340,3 +340,112 @@ int lq_oracle_w4a8_gemm_sampled(const int8_t* x_q, const float* s_x, const uint8
   if (bad & 4) return ORC_ERR_INT32_RANGE;
   return ORC_OK;
 }
+
+/* ====================================================================== */
+/* W4 x FP8 variant (FireQ page, abstract: INT4 weights with channel-wise  */
+/* scaling, FP8 activations with a per-tensor scale).  The pages give no   */
+/* formulas; the readings used here:                                       */
+/*   weights:     s_w[n] = amax_n / 7, q = clamp(rint(w * (7 / amax_n)),   */
+/*                -7, 7), stored as u = q + 8 in the LiquidQuant nibble    */
+/*                layout; a zero row gets s_w = 1 and q = 0;               */
+/*   activations: one scale for the tensor, s_x = amax / 448 (448 is the   */
+/*                largest finite e4m3 value), codes e4m3(x * (448 / amax)) */
+/*                rounded to nearest even and saturated to +-448; a zero   */
+/*                tensor gets s_x = 1;                                     */
+/*   GEMM:        acc[m,n] = sum_k e4m3(x)[m,k] * q[n,k], exact (every     */
+/*                product and partial sum is a multiple of 2^-9 far below  */
+/*                2^53 in magnitude, so double holds it exactly), then     */
+/*                out = bf16((float)acc * (s_x * s_w[n])).                 */
+/* ====================================================================== */
+
+/* e4m3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent    */
+/* field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; no infinities; the   */
+/* largest finite value is 1.75 * 2^8 = 448.                                 */
+float lq_oracle_e4m3_to_f32(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  const float v = e == 0 ? ldexpf((float)m, -9) : ldexpf(1.0f + (float)m / 8.0f, e - 7);
+  return s ? -v : v;
+}
+
+/* Round to nearest even, saturating finite values beyond 448 to 448. */
+uint8_t lq_oracle_f32_to_e4m3(float x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const float a = fabsf(x);
+  if (a >= 448.0f) return sign | 0x7E;
+  int e2;
+  frexpf(a, &e2);               /* a = f * 2^e2, f in [0.5, 1): floor(log2 a) = e2 - 1 */
+  int E = (a == 0.0f) ? 1 : (e2 - 1) + 7;
+  if (E < 1) E = 1;             /* the subnormal range shares exponent field 1's quantum */
+  const float quantum = ldexpf(1.0f, E - 7 - 3);
+  const int n = (int)nearbyintf(a / quantum);  /* a / quantum is exact (power-of-two quantum) */
+  /* n in [0, 16]: below 8 only in the subnormal range; 16 carries into the next binade */
+  int code;
+  if (n < 8)
+    code = n;                       /* subnormal (E == 1 here) */
+  else if (n == 16)
+    code = ((E + 1) << 3);          /* E + 1 <= 15: a < 448 never rounds past 448 */
+  else
+    code = (E << 3) | (n - 8);
+  return sign | (uint8_t)code;
+}
+
+int lq_oracle_quantize_weights_w4(const uint16_t* W, int N, int K, uint8_t* qw4, float* s_w) {
+  if (!W || !qw4 || !s_w || N < 0 || K < 0 || K % 8 != 0) return ORC_ERR_ARG;
+  for (int n = 0; n < N; ++n) {
+    const uint16_t* row = W + (size_t)n * K;
+    float amax = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      float a = fabsf(bf16_to_f32(row[k]));
+      if (a > amax) amax = a;
+    }
+    const float inv = amax == 0.0f ? 0.0f : 7.0f / amax;
+    s_w[n] = amax == 0.0f ? 1.0f : amax / 7.0f;
+    uint8_t* prow = qw4 + (size_t)n * (K / 2);
+    memset(prow, 0, (size_t)K / 2);
+    for (int k = 0; k < K; ++k) {
+      const int q = amax == 0.0f ? 0 : clampi((int)nearbyintf(bf16_to_f32(row[k]) * inv), -7, 7);
+      const int u = q + 8;
+      const int j = k / 8, r = k % 8;       /* word j, code r: byte r%4, high nibble if r >= 4 */
+      prow[4 * j + (r & 3)] |= (uint8_t)(r < 4 ? u : u << 4);
+    }
+  }
+  return ORC_OK;
+}
+
+int lq_oracle_quantize_act_f8(const uint16_t* X, int M, int K, uint8_t* x_f8, float* s_x) {
+  if (!X || !x_f8 || !s_x || M < 0 || K < 0) return ORC_ERR_ARG;
+  float amax = 0.0f;
+  for (size_t i = 0; i < (size_t)M * K; ++i) {
+    float a = fabsf(bf16_to_f32(X[i]));
+    if (a > amax) amax = a;
+  }
+  const float inv = amax == 0.0f ? 0.0f : 448.0f / amax;
+  *s_x = amax == 0.0f ? 1.0f : amax / 448.0f;
+  for (size_t i = 0; i < (size_t)M * K; ++i) x_f8[i] = lq_oracle_f32_to_e4m3(bf16_to_f32(X[i]) * inv);
+  return ORC_OK;
+}
+
+int lq_oracle_w4f8_gemm(const uint8_t* x_f8, float s_x, const uint8_t* qw4, const float* s_w, int M, int N, int K,
+                        uint16_t* out, double* acc_out) {
+  if (!x_f8 || !qw4 || !s_w || !out || M < 0 || N < 0 || K < 0 || K % 8 != 0) return ORC_ERR_ARG;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : bad)
+  for (int n = 0; n < N; ++n) {
+    const uint8_t* prow = qw4 + (size_t)n * (K / 2);
+    for (int m = 0; m < M; ++m) {
+      const uint8_t* xr = x_f8 + (size_t)m * K;
+      double s = 0.0;
+      for (int k = 0; k < K; ++k) {
+        const float xv = lq_oracle_e4m3_to_f32(xr[k]);
+        if (isnan(xv)) bad |= 1;
+        const int u = unpack_code(prow, k);
+        s += (double)xv * (double)(u - 8);
+      }
+      if (acc_out) acc_out[(size_t)m * N + n] = s;
+      out[(size_t)m * N + n] = f32_to_bf16_rne((float)s * (s_x * s_w[n]));
+    }
+  }
+  return bad ? ORC_ERR_ARG : ORC_OK;
+}

@@ -377,3 +377,104 @@ def test_grouped_gemm_against_float64_rows():
     o2, a2 = oracle.w4a8_gemm(x_q, s_x, qw[:N], s_u8[:, :N], a_u8[:, :N], s_c[:N])
     np.testing.assert_array_equal(a1, a2)
     np.testing.assert_array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------------------
+# W4 x FP8 variant: e4m3 against torch's float8_e4m3fn (a library routine),
+# the INT4 and FP8 quantizers against their closed forms, the GEMM against a
+# float64 product of the decoded operands
+# ---------------------------------------------------------------------------
+
+def _torch_e4m3_code(x: float) -> int:
+    return int(torch.tensor([x], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+
+
+def test_e4m3_decode_all_codes_match_torch():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).float().numpy()
+    got = np.array([oracle.e4m3_to_f32(c) for c in range(256)], np.float32)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok].view(np.uint32), ref[ok].view(np.uint32))
+    assert oracle.e4m3_to_f32(0x7E) == 448.0 and oracle.e4m3_to_f32(0x01) == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_rounding_and_saturates():
+    # every bf16 value: round to nearest even wherever torch's conversion is finite
+    bits = np.arange(65536, dtype=np.uint32) << 16
+    vals = bits.view(np.float32)
+    fin = np.isfinite(vals) & (np.abs(vals) <= 464.0)
+    ref = torch.from_numpy(vals[fin].copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.f32_to_e4m3(v) for v in vals[fin]], np.uint8)
+    np.testing.assert_array_equal(got, ref)
+    # ties between neighbouring codes go to the even code, as in torch
+    for c in range(0x7E):
+        lo, hi = oracle.e4m3_to_f32(c), oracle.e4m3_to_f32(c + 1)
+        mid = np.float32((lo + hi) / 2)
+        assert oracle.f32_to_e4m3(mid) == _torch_e4m3_code(float(mid)) == (c if c % 2 == 0 else c + 1)
+        assert oracle.f32_to_e4m3(-mid) == 0x80 | (c if c % 2 == 0 else c + 1)
+    # finite values beyond the largest code saturate to +-448 (torch gives NaN there)
+    for x in (465.0, 500.0, 1e6, 3.4e38):
+        assert oracle.f32_to_e4m3(x) == 0x7E and oracle.f32_to_e4m3(-x) == 0xFE
+    assert oracle.f32_to_e4m3(float("nan")) == 0x7F
+
+
+def test_w4_weight_quantizer_closed_form():
+    from w4a8_bit_weight_b200 import synth
+    _, W = synth.make_problem(1, 48, 256, seed=12, n_outliers=0)
+    W[5] = 0
+    wb = synth.bf16_bits(W)
+    qw4, s_w = oracle.quantize_weights_w4(wb)
+    w = W.float().numpy()
+    u = np.empty(w.shape, np.int64)
+    u[:, 0::8], u[:, 4::8] = (qw4[:, 0::4] & 15), (qw4[:, 0::4] >> 4)
+    u[:, 1::8], u[:, 5::8] = (qw4[:, 1::4] & 15), (qw4[:, 1::4] >> 4)
+    u[:, 2::8], u[:, 6::8] = (qw4[:, 2::4] & 15), (qw4[:, 2::4] >> 4)
+    u[:, 3::8], u[:, 7::8] = (qw4[:, 3::4] & 15), (qw4[:, 3::4] >> 4)
+    q = u - 8
+    assert q.min() >= -7 and q.max() <= 7
+    amax = np.abs(w).max(axis=1)
+    for n in range(w.shape[0]):
+        if amax[n] == 0:
+            assert s_w[n] == 1.0 and (q[n] == 0).all()
+            continue
+        assert s_w[n] == np.float32(amax[n]) / np.float32(7.0)
+        inv = np.float32(7.0) / np.float32(amax[n])
+        np.testing.assert_array_equal(q[n], np.clip(np.rint((w[n] * inv).astype(np.float32)), -7, 7))
+        assert np.abs(q[n][np.argmax(np.abs(w[n]))]) == 7
+        assert np.all(np.abs(w[n] - q[n] * s_w[n]) <= s_w[n] * 0.5 * (1 + 1e-5))
+
+
+def test_f8_activation_quantizer_closed_form():
+    from w4a8_bit_weight_b200 import synth
+    X, _ = synth.make_problem(6, 16, 128, seed=13, n_outliers=2)
+    xb = synth.bf16_bits(X)
+    x_f8, s_x = oracle.quantize_act_f8(xb)
+    x = X.float().numpy()
+    amax = np.float32(np.abs(x).max())
+    assert s_x == amax / np.float32(448.0)
+    inv = np.float32(448.0) / amax
+    ref = torch.from_numpy((x * inv).astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(x_f8, ref)
+    assert (x_f8 & 0x7F).max() == 0x7E       # the largest |x| maps to 448
+    z, sz = oracle.quantize_act_f8(np.zeros((2, 64), np.uint16))
+    assert sz == 1.0 and not z.any()
+
+
+def test_w4f8_gemm_exact_against_float64():
+    from w4a8_bit_weight_b200 import synth
+    X, W = synth.make_problem(9, 40, 512, seed=14, n_outliers=3)
+    qw4, s_w = oracle.quantize_weights_w4(synth.bf16_bits(W))
+    x_f8, s_x = oracle.quantize_act_f8(synth.bf16_bits(X))
+    out, acc = oracle.w4f8_gemm(x_f8, s_x, qw4, s_w)
+    xv = torch.from_numpy(x_f8.copy()).view(torch.float8_e4m3fn).double().numpy()
+    u = np.stack([(qw4 >> (4 * h)) & 15 for h in (0, 1)], -1)            # [N, K/2, 2]: low, high nibble
+    u = u.reshape(qw4.shape[0], -1, 4, 2).transpose(0, 1, 3, 2).reshape(qw4.shape[0], -1)
+    q = u.astype(np.float64) - 8
+    np.testing.assert_array_equal(acc, xv @ q.T)
+    y = torch.from_numpy(acc.astype(np.float32)) * (torch.tensor(s_x) * torch.from_numpy(s_w))
+    np.testing.assert_array_equal(out, y.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    # a real approximation of the bf16 product: 7 levels per sign per channel, FP8 activations
+    ref = X.double().numpy() @ W.double().numpy().T
+    got = torch.from_numpy(out.view(np.int16)).view(torch.bfloat16).double().numpy()
+    assert np.sqrt(np.mean((got - ref) ** 2)) < 0.35 * np.std(ref)
