@@ -270,6 +270,16 @@ LQ_API lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const
                                       void* out_bf16, int M, int N, int K, int group, void* stream);
 
 /*
+ * lq_plan_gemm -- TEST ONLY, touches no device: the schedule lq_w4a8_gemm_ex
+ * would run for these arguments on a GPU with `sms` multiprocessors.  On
+ * LQ_OK, plan[0..3] = schedule kind (LQ_SCHED_*), token-tile width, CTAs per
+ * cluster (0 for stream-K, 2 for CTA pairs), grid size.  Argument errors as
+ * in lq_w4a8_gemm_ex (M >= 1 here).
+ */
+LQ_API lq_status lq_plan_gemm(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms,
+                              int* plan);
+
+/*
  * lq_w4a8_gemm_ablation -- TEST AND MEASUREMENT ONLY: the pages' ablation of
  * the dequantization arithmetic (LQQ) and of the pipeline (explicit
  * coarse-grained, ExCP, vs implicit fine-grained, ImFP: LiquidGEMM Figs. 6

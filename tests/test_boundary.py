@@ -172,3 +172,38 @@ def test_ablation_rejects_before_launch(lib):
     assert call(bt=32) == 2 and call(bt=128) == 2 and call(split=2) == 2
     assert call(K=192) == 2 and call(x=ODD) == 3 and call(out=P(0)) == 1
     assert call(M=0) == 0
+
+
+def _plan(lib, M, N, K, sms=148, bt=0, sched=0, split=0, grid=0):
+    out = (ctypes.c_int * 4)()
+    st = lib.lq_plan_gemm(M, N, K, bt, sched, split, grid, sms, out)
+    return st, tuple(out)
+
+
+@pytest.mark.parametrize("M,N,K,plan", [
+    # (kind, token tile, CTAs per cluster, grid) on 148 SMs; kinds: 1 tiles, 2 persistent, 4 CTA pairs
+    (16, 4096, 4096, (1, 16, 4, 128)),       # decode: 4-CTA clusters, one wave
+    (1, 4096, 14336, (1, 16, 8, 256)),       # long K-slices: 8-CTA clusters, two CTAs per SM
+    (32, 4096, 14336, (1, 32, 8, 256)),      # 32-token tiles in 8-CTA clusters fit two per SM (7 stages)
+    (64, 4096, 14336, (1, 64, 4, 128)),      # 64-token tiles: 4-CTA clusters, one per SM
+    (128, 4096, 14336, (1, 128, 4, 128)),    # 128-token tiles in 4-CTA clusters
+    (256, 4096, 14336, (1, 128, 2, 128)),    # 16 pair tiles: too few for pairs; 64 tiles, 2-CTA clusters
+    (16, 14336, 4096, (1, 16, 2, 224)),      # 112 tiles: 2-CTA clusters, two per SM
+    (128, 14336, 4096, (1, 128, 1, 112)),    # at most 128 tokens: never pairs
+    (256, 14336, 4096, (4, 256, 2, 112)),    # 56 pair tiles >= 148 / 4: CTA pairs
+    (1024, 4096, 14336, (4, 256, 2, 128)),   # 64 pair tiles: 64 pairs
+    (4096, 4096, 4096, (4, 256, 2, 148)),    # prefill: 74 persistent pairs
+    (4096, 4096, 384, (2, 128, 1, 148)),     # K not a multiple of 256: persistent 128-token tiles
+])
+def test_automatic_schedule(lib, M, N, K, plan):
+    st, got = _plan(lib, M, N, K)
+    assert st == 0 and got == plan, got
+
+
+def test_plan_follows_explicit_choices(lib):
+    assert _plan(lib, 16, 256, 1024, bt=16, sched=1, split=2) == (0, (1, 16, 2, 4))
+    assert _plan(lib, 16, 256, 1024, bt=16, sched=3, grid=3) == (0, (3, 16, 0, 3))
+    assert _plan(lib, 512, 512, 2048, sched=4, grid=2) == (0, (4, 256, 2, 2))
+    assert _plan(lib, 16, 256, 1024, bt=64, sched=1, split=8)[0] == 1     # split 8 needs <= 32 tokens
+    assert _plan(lib, 300, 256, 384, sched=4)[0] == 2                     # pairs need K % 256 == 0
+    assert _plan(lib, 16, 4096, 4096, sms=0)[0] == 1

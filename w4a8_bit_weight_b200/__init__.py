@@ -78,6 +78,7 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_grouped_gemm": ([P, P, P, P, P, P, P, I, P, I, I, I, I, P], I),
             "lq_w4a8_gemm_ablation": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P], I),
             "lq_test_wait_timeout": ([P], I),
+            "lq_plan_gemm": ([I, I, I, I, I, I, I, I, P], I),
             "lq_w4a8_grouped_gemm_ex": ([P, P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():

@@ -648,6 +648,21 @@ lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* 
                    0, 0, 0, true, stream);
 }
 
+lq_status lq_plan_gemm(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms, int* plan) {
+  if (!plan || sms < 1) return LQ_ERR_INVALID_ARG;
+  lq_status st = check_gemm_shape(M, N, K, LQ_GROUP);
+  if (st != LQ_OK) return st;
+  if (M < 1 || !valid_schedule(M, block_t, schedule, split_k, grid)) return LQ_ERR_INVALID_ARG;
+  const Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, sms);
+  st = check_schedule_shape(s, K);
+  if (st != LQ_OK) return st;
+  plan[0] = s.kind;
+  plan[1] = s.bt;
+  plan[2] = s.cs;
+  plan[3] = s.grid;
+  return LQ_OK;
+}
+
 lq_status lq_w4a8_gemm_ablation(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                                 const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
                                 int variant, int block_t, int split_k, int out_i32, void* stream) {
