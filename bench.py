@@ -435,6 +435,10 @@ def run_ours(args, rank, world, local_rank):
         res["prefill"] = pre
         res["grouped"] = grouped_side(dev, int8_peak, hbm_peak)
         res["ablation"] = ablation_side(dev, hbm_peak)
+        try:
+            res["w4f8"] = w4f8_side(dev, hbm_peak)
+        except Exception as ex:  # a side measurement never takes the bench line down
+            res["w4f8"] = {"error": str(ex)[:200]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w)
     return res
@@ -557,6 +561,50 @@ def ablation_side(dev, hbm_peak, n=40):
             entry[nm]["slowdown_vs_lqq_implicit"] = entry[nm]["us"] / base
         res[label] = entry
         del sets, qw, s_u8, a_u8, s_c
+    return res
+
+
+def w4f8_side(dev, hbm_peak, n=40):
+    """The W4 x FP8 variant on the decode layer (N = K = 4096, M = 1, 4, 16): n back-to-back
+    lq_w4f8_gemm calls per M in one CUDA graph, weights rotating over L2-cold copies."""
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+    w = synth.WORKLOADS["decode"]
+    X, W = synth.make_workload(w)
+    qw4, s_w = lq.lq_quantize_weights_w4(W.to(dev))
+    wset = qw4.numel() + 4 * s_w.numel()
+    n_sets = min(48, max(4, int(np.ceil(3 * L2_BYTES / wset))))
+    sets = [(qw4, s_w)] + [(qw4.clone(), s_w.clone()) for _ in range(n_sets - 1)]
+    stream = torch.cuda.Stream(dev)
+    res = {"workload": w.note, "how": f"{n} back-to-back lq_w4f8_gemm calls per M in one CUDA graph; "
+                                      "bytes = INT4 weights + s_w + e4m3 x + s_x + bf16 out"}
+    Xd = X.to(dev)
+    for M in w.Ms:
+        x_f8, s_x = lq.lq_quantize_act_f8(Xd[:M])
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
+        with torch.cuda.stream(stream):
+            for i in range(2):
+                lq.lq_w4f8_gemm(x_f8, s_x, *sets[i % n_sets], out=out)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    lq.lq_w4f8_gemm(x_f8, s_x, *sets[i % n_sets], out=out)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            ts = []
+            for _ in range(3):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(1e3 * e0.elapsed_time(e1) / n)
+        if lq.lq_get_device_error(dev) != 0:
+            raise RuntimeError("device error in the W4 x FP8 measurement")
+        us = sorted(ts)[1]
+        byts = w.N * w.K // 2 + 4 * w.N + M * w.K + 4 + 2 * M * w.N
+        res[str(M)] = {"us": us, "gbs": byts / (us * 1e-6) / 1e9, "frac_of_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
+        del g
     return res
 
 

@@ -351,6 +351,30 @@ LQ_API lq_status lq_w4a8_grouped_gemm_ex(const int8_t* x_q, const float* s_x, co
                                          int group, int block_t, int split_k, int out_i32, void* stream);
 
 /*
+ * The W4 x FP8 variant (FireQ page, abstract: INT4 weights with channel-wise
+ * scaling, FP8 activations with one scale for the tensor).  The pages give
+ * no formulas; the readings:
+ * lq_quantize_weights_w4 -- per-channel symmetric INT4: s_w[n] = amax_n / 7,
+ *   q = clamp(rint(w * (7 / amax_n)), -7, 7) with IEEE fp32 operations,
+ *   stored as q + 8 in the LiquidQuant nibble layout (qw4 [N, K/2]); a zero
+ *   row gets s_w = 1 and q = 0.  K % 16 == 0; W and qw4 16-byte aligned.
+ * lq_quantize_act_f8 -- FP8 e4m3 activations with one scale for the tensor:
+ *   s_x[0] = amax / 448, x_f8 = e4m3(x * (448 / amax)), round to nearest
+ *   even, saturated to +-448 (cvt ... satfinite); an all-zero or empty
+ *   tensor gets s_x = 1.  Three launches and a 4-byte memset on `stream`
+ *   (the tensor's maximum is gathered in s_x's word first).  K % 16 == 0.
+ * lq_w4f8_gemm -- out[m,n] = bf16(acc * (s_x[0] * s_w[n])), acc the fp32
+ *   sum over k of e4m3(x)[m,k] * q[n,k] computed by tcgen05.mma
+ *   kind::f8f6f4 (the products are exact, the fp32 accumulation order is the
+ *   tensor core's).  One CTA per 128-row x 16- or 128-token tile.  Shape and
+ *   alignment rules as lq_w4a8_gemm (no group, no workspace).
+ */
+LQ_API lq_status lq_quantize_weights_w4(const void* W_bf16, int N, int K, uint8_t* qw4, float* s_w, void* stream);
+LQ_API lq_status lq_quantize_act_f8(const void* X_bf16, int M, int K, uint8_t* x_f8, float* s_x, void* stream);
+LQ_API lq_status lq_w4f8_gemm(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4, const float* s_w,
+                              void* out_bf16, int M, int N, int K, void* stream);
+
+/*
  * lq_test_wait_timeout -- TEST ONLY: launches a one-CTA kernel whose first
  * warp waits on an mbarrier that nothing completes, with the GEMM kernels'
  * bounded wait: after the 2 s limit it raises the CTA's abort flag and

@@ -79,6 +79,9 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_gemm_ablation": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P], I),
             "lq_test_wait_timeout": ([P], I),
             "lq_plan_gemm": ([I, I, I, I, I, I, I, I, P], I),
+            "lq_quantize_weights_w4": ([P, I, I, P, P, P], I),
+            "lq_quantize_act_f8": ([P, I, I, P, P, P], I),
+            "lq_w4f8_gemm": ([P, P, P, P, P, I, I, I, P], I),
             "lq_w4a8_grouped_gemm_ex": ([P, P, P, P, P, P, P, I, P, I, I, I, I, I, I, I, P], I),
         }
         for name, (args, res) in sig.items():
@@ -374,6 +377,50 @@ def lq_dequant_weights_i8(qw, s_u8, a_u8, group: int = GROUP, out=None):
     with torch.cuda.device(qw.device):
         _check("lq_dequant_weights_i8", lib.lq_dequant_weights_i8(
             _ptr(qw), _ptr(s_u8), _ptr(a_u8), N, K, group, _ptr(out), _stream(qw.device)))
+    return out
+
+
+def lq_quantize_weights_w4(W: torch.Tensor, out=None):
+    """W4 x FP8 variant: per-channel symmetric INT4 weights -> (qw4 [N, K/2] uint8, s_w [N] fp32)."""
+    lib = load_library()
+    _need(W, torch.bfloat16, "W")
+    N, K = W.shape
+    qw4, s_w = out if out is not None else (torch.empty(N, K // 2, dtype=torch.uint8, device=W.device),
+                                            torch.empty(N, dtype=torch.float32, device=W.device))
+    with torch.cuda.device(W.device):
+        _check("lq_quantize_weights_w4", lib.lq_quantize_weights_w4(_ptr(W), N, K, _ptr(qw4), _ptr(s_w),
+                                                                    _stream(W.device)))
+    return qw4, s_w
+
+
+def lq_quantize_act_f8(X: torch.Tensor, out=None):
+    """W4 x FP8 variant: e4m3 codes with one scale for the tensor -> (x_f8 [M, K] uint8, s_x [1] fp32)."""
+    lib = load_library()
+    _need(X, torch.bfloat16, "X")
+    M, K = X.shape
+    x_f8, s_x = out if out is not None else (torch.empty(M, K, dtype=torch.uint8, device=X.device),
+                                             torch.empty(1, dtype=torch.float32, device=X.device))
+    with torch.cuda.device(X.device):
+        _check("lq_quantize_act_f8", lib.lq_quantize_act_f8(_ptr(X), M, K, _ptr(x_f8), _ptr(s_x),
+                                                            _stream(X.device)))
+    return x_f8, s_x
+
+
+def lq_w4f8_gemm(x_f8, s_x, qw4, s_w, out=None):
+    """W4 x FP8 GEMM: bf16(fp32 sum_k e4m3(x) * q * s_x * s_w[n]) -> [M, N] bf16."""
+    lib = load_library()
+    _need(x_f8, torch.uint8, "x_f8")
+    M, K = x_f8.shape
+    N = qw4.shape[0]
+    _need(qw4, torch.uint8, "qw4", (N, K // 2))
+    _need(s_x, torch.float32, "s_x", (1,))
+    _need(s_w, torch.float32, "s_w", (N,))
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=x_f8.device)
+    _need(out, torch.bfloat16, "out", (M, N))
+    with torch.cuda.device(x_f8.device):
+        _check("lq_w4f8_gemm", lib.lq_w4f8_gemm(_ptr(x_f8), _ptr(s_x), _ptr(qw4), _ptr(s_w), _ptr(out), M, N, K,
+                                                _stream(x_f8.device)))
     return out
 
 

@@ -14,6 +14,7 @@
 #include "../../include/lq.h"
 #include "lq_device.cuh"
 #include "lq_gemm_kernel.cuh"
+#include "lq_gemm_w4f8.cuh"
 #include "lq_gemm_persistent.cuh"
 #include "lq_gemm_pair.cuh"
 #include "lq_quant_kernels.cuh"
@@ -875,6 +876,88 @@ lq_status lq_w4a8_grouped_gemm(const int8_t* x_q, const float* s_x, const uint8_
                                const uint8_t* a_u8, const float* s_c, const int* m_off, int groups, void* out_bf16,
                                int M, int N, int K, int group, void* stream) {
   return grouped_impl(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, groups, out_bf16, M, N, K, group, 0, 0, false, stream);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------ W4 x FP8
+extern "C" {
+
+lq_status lq_quantize_weights_w4(const void* W_bf16, int N, int K, uint8_t* qw4, float* s_w, void* stream) {
+  if (N < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (K < 16 || K % 16 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return LQ_OK;
+  if (!W_bf16 || !qw4 || !s_w) return LQ_ERR_INVALID_ARG;
+  if (!aligned(W_bf16, 16) || !aligned(qw4, 16) || !aligned(s_w, 4)) return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  const lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  lq::quantize_weights_w4_kernel<<<N, lq::kW4Threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W_bf16), K, qw4, s_w);
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+lq_status lq_quantize_act_f8(const void* X_bf16, int M, int K, uint8_t* x_f8, float* s_x, void* stream) {
+  if (M < 0 || K < 0) return LQ_ERR_INVALID_ARG;
+  if (K < 16 || K % 16 != 0) return LQ_ERR_UNSUPPORTED_SHAPE;
+  if (!s_x || (M > 0 && (!X_bf16 || !x_f8))) return LQ_ERR_INVALID_ARG;
+  if ((M > 0 && (!aligned(X_bf16, 16) || !aligned(x_f8, 16))) || !aligned(s_x, 4)) return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  const lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // the tensor's amax in s_x's word, the codes, then s_x itself (an empty tensor gets s_x = 1)
+  if (cudaMemsetAsync(s_x, 0, sizeof(float), cs) != cudaSuccess) return LQ_ERR_CUDA;
+  unsigned int* amax_bits = reinterpret_cast<unsigned int*>(s_x);
+  if (M > 0) {
+    lq::act_f8_amax_kernel<<<M, lq::kQuantActThreads, 0, cs>>>(static_cast<const uint16_t*>(X_bf16), K, amax_bits);
+    lq::act_f8_codes_kernel<<<M, lq::kQuantActThreads, 0, cs>>>(static_cast<const uint16_t*>(X_bf16), K, amax_bits,
+                                                                 x_f8);
+  }
+  lq::act_f8_scale_kernel<<<1, 1, 0, cs>>>(s_x);
+  return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+lq_status lq_w4f8_gemm(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4, const float* s_w, void* out_bf16,
+                       int M, int N, int K, void* stream) {
+  lq_status st = check_gemm_shape(M, N, K, LQ_GROUP);
+  if (st != LQ_OK) return st;
+  if (M == 0) return LQ_OK;
+  if (!x_f8 || !s_x || !qw4 || !s_w || !out_bf16) return LQ_ERR_INVALID_ARG;
+  if (!aligned(x_f8, 16) || !aligned(qw4, 16) || !aligned(out_bf16, 16) || !aligned(s_x, 4) || !aligned(s_w, 4))
+    return LQ_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  const int bt = M <= 16 ? 16 : 128;
+  const int tiles_m = (M + bt - 1) / bt, tiles_n = (N + lq::kBlockN - 1) / lq::kBlockN;
+  if ((long long)tiles_m * tiles_n > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tx, tw;
+  if (!make_map_u8(&tx, x_f8, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128u, (uint32_t)bt, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&tw, qw4, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 64u, 128u, CU_TENSOR_MAP_SWIZZLE_64B))
+    return LQ_ERR_CUDA;
+  lq::F8Args a;
+  a.s_x = s_x;
+  a.s_w = s_w;
+  a.out = static_cast<__nv_bfloat16*>(out_bf16);
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = tiles_m;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int grid = tiles_m * tiles_n;
+  if (bt == 16) {
+    auto kern = lq::w4f8_gemm_kernel<16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::F8Cfg<16>::kSmemBytes) !=
+        cudaSuccess)
+      return LQ_ERR_CUDA;
+    return launch_ex(kern, grid, lq::kF8Threads, lq::F8Cfg<16>::kSmemBytes, 1, pdl_enabled(), cs, tx, tw, a);
+  }
+  auto kern = lq::w4f8_gemm_kernel<128>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::F8Cfg<128>::kSmemBytes) !=
+      cudaSuccess)
+    return LQ_ERR_CUDA;
+  return launch_ex(kern, grid, lq::kF8Threads, lq::F8Cfg<128>::kSmemBytes, 1, pdl_enabled(), cs, tx, tw, a);
 }
 
 }  // extern "C"
