@@ -207,3 +207,23 @@ def test_plan_follows_explicit_choices(lib):
     assert _plan(lib, 16, 256, 1024, bt=64, sched=1, split=8)[0] == 1     # split 8 needs <= 32 tokens
     assert _plan(lib, 300, 256, 384, sched=4)[0] == 2                     # pairs need K % 256 == 0
     assert _plan(lib, 16, 4096, 4096, sms=0)[0] == 1
+
+
+def test_w4f8_entry_points_reject_before_launch(lib):
+    qw = lib.lq_quantize_weights_w4
+    assert qw(GOOD, 16, 192 + 8, GOOD, GOOD, None) == 2      # K % 16
+    assert qw(GOOD, -1, 256, GOOD, GOOD, None) == 1
+    assert qw(None, 16, 256, GOOD, GOOD, None) == 1
+    assert qw(ODD, 16, 256, GOOD, GOOD, None) == 3
+    assert qw(None, 0, 256, None, None, None) == 0           # no rows: nothing to do
+    qa = lib.lq_quantize_act_f8
+    assert qa(GOOD, 4, 100, GOOD, GOOD, None) == 2
+    assert qa(GOOD, 4, 256, GOOD, None, None) == 1            # s_x always written
+    assert qa(ODD, 4, 256, GOOD, GOOD, None) == 3
+    assert qa(GOOD, 4, 256, GOOD, P((1 << 20) + 2), None) == 3
+    g = lib.lq_w4f8_gemm
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, 16, 200, 512, None) == 2   # N % 16
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, 16, 256, 192, None) == 2   # K % 128
+    assert g(GOOD, None, GOOD, GOOD, GOOD, 16, 256, 512, None) == 1
+    assert g(GOOD, GOOD, GOOD, GOOD, ODD, 16, 256, 512, None) == 3
+    assert g(None, None, None, None, None, 0, 256, 512, None) == 0    # empty batch
