@@ -227,3 +227,33 @@ def test_w4f8_entry_points_reject_before_launch(lib):
     assert g(GOOD, None, GOOD, GOOD, GOOD, 16, 256, 512, None) == 1
     assert g(GOOD, GOOD, GOOD, GOOD, ODD, 16, 256, 512, None) == 3
     assert g(None, None, None, None, None, 0, 256, 512, None) == 0    # empty batch
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """include/lq.h compiles as strict C99, and a C program linked against the library
+    calls it without Python (the calls used touch no device)."""
+    import os
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_lq.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "lq.h"\n'
+        "int main(void) {\n"
+        "  int plan[4];\n"
+        "  if (lq_version() < 100) return 1;\n"
+        "  if (lq_plan_gemm(16, 4096, 4096, 0, LQ_SCHED_AUTO, 0, 0, 148, plan) != LQ_OK) return 2;\n"
+        "  if (plan[0] != LQ_SCHED_TILES || plan[1] != 16 || plan[2] != 4) return 3;\n"
+        "  if (lq_w4a8_gemm_workspace_size(16, 4096, 4096) != 0) return 4;\n"
+        '  printf("%s\\n", lq_status_string(LQ_ERR_WORKSPACE));\n'
+        "  return 0;\n}\n")
+    libdir = os.path.join(root, "w4a8_bit_weight_b200")
+    exe = tmp_path / "use_lq"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+                    str(src), "-L", libdir, "-llq_b200", "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.strip().startswith(lq.STATUS[4])
