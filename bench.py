@@ -14,8 +14,10 @@ events on the launching stream, after W warm-up steps and about a second of
 untimed replays (so the clock sampler sees the GPU under load).  Each GEMM
 launch reads a different copy of the layer's packed weights, rotating over
 enough copies that the working set is several times the 126 MB L2, so every
-launch streams its weights from HBM.  External CUDA events around every GEMM
-node give the GEMM's own average duration for the roofline.
+launch streams its weights from HBM.  The GEMM's own duration per launch (the
+roofline's denominator) comes from a second graph of K back-to-back GEMM calls
+per M, timed the same way: the launches overlap through programmatic dependent
+launch exactly as in the step, and replay time / K is the time per launch.
 
 With --gpus N > 1 (launched by torchrun) every rank runs an independent
 replica (the path has no exchange step); the time is the max over ranks and

@@ -257,3 +257,25 @@ def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stderr)
     assert r.stdout.strip().startswith(lq.STATUS[4])
+
+
+def test_timeout_status_clears_cached_workspaces():
+    """After LQ_ERR_TIMEOUT a stream-K call may have left partial sums in its workspace:
+    the binding zeroes every cached GEMM workspace (and only those)."""
+    import torch
+    import w4a8_bit_weight_b200 as lq
+    saved = dict(lq._ws)
+    try:
+        lq._ws.clear()
+        gemm_ws = torch.full((64,), 7, dtype=torch.uint8)
+        lin_ws = torch.full((64,), 9, dtype=torch.uint8)
+        lq._ws[("gemm", 0)] = gemm_ws
+        lq._ws[("linear", 0)] = lin_ws
+        lq._after_device_error(0)
+        assert int(gemm_ws.min()) == 7
+        lq._after_device_error(lq.LQ_ERR_TIMEOUT)
+        assert not gemm_ws.any()
+        assert int(lin_ws.min()) == 9  # lq_w4a8_linear's front holds x_q / s_x, not sums
+    finally:
+        lq._ws.clear()
+        lq._ws.update(saved)

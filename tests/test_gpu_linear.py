@@ -79,6 +79,17 @@ def test_linear_matches_two_step_and_oracle(M, N, K, fusable):
     if M * N * K <= 16 * 4096 * 4096:
         o_out, _ = oracle.w4a8_gemm(o_xq, o_sx, o_qw, o_s, o_a, o_sc)
         assert int(_ulps(_u16(out), o_out).max()) <= 1
+    else:
+        # larger layers: every tile corner and ragged edge plus 20000 random outputs,
+        # each computed by the oracle on its own
+        rng = np.random.default_rng(M + N + K)
+        edge_m = sorted({0, M - 1} | {m for m in (15, 16) if m < M})
+        edge_n = sorted({0, N - 1} | {n for n in range(127, N, 128)} | {n for n in range(128, N, 128)})
+        mi = [m for m in edge_m for _ in edge_n] + rng.integers(0, M, 20000).tolist()
+        ni = [n for _ in edge_m for n in edge_n] + rng.integers(0, N, 20000).tolist()
+        mi, ni = np.array(mi, np.int64), np.array(ni, np.int64)
+        o_out, _ = oracle.w4a8_gemm_sampled(o_xq, o_sx, o_qw, o_s, o_a, o_sc, mi, ni)
+        assert int(_ulps(_u16(out)[mi, ni], o_out).max()) <= 1
     if M >= 3:
         assert not (_u16(out)[2] & 0x7FFF).any()
 

@@ -234,7 +234,7 @@ def _sample_points(M, N, n_rand, seed):
     return np.array(mi, np.int64), np.array(ni, np.int64)
 
 
-def _workload_check(name, Ms, full_limit=4 * 10 ** 8, n_rand=3000):
+def _workload_check(name, Ms, full_limit=4 * 10 ** 8, n_rand=20000):
     w = synth.WORKLOADS[name]
     X, W = synth.make_workload(w)
     Wd = W.to(DEV)
@@ -281,4 +281,4 @@ def test_workload_mlp_up():
 
 
 def test_workload_down_sweep():
-    _workload_check("down_sweep", synth.WORKLOADS["down_sweep"].Ms, n_rand=1500)
+    _workload_check("down_sweep", synth.WORKLOADS["down_sweep"].Ms)

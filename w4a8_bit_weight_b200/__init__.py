@@ -432,12 +432,28 @@ def lq_test_wait_timeout(device=None) -> None:
         _check("lq_test_wait_timeout", lib.lq_test_wait_timeout(_stream(dev)))
 
 
+LQ_ERR_TIMEOUT = 6
+
+
+def _after_device_error(status: int) -> None:
+    """A kernel that gave up a wait (LQ_ERR_TIMEOUT) may have left partial sums
+    and tile tickets in a stream-K workspace, which the kernels otherwise restore
+    to zero: clear every cached GEMM workspace so that later calls start clean."""
+    if status == LQ_ERR_TIMEOUT:
+        for (kind, _), buf in _ws.items():
+            if kind == "gemm":
+                buf.zero_()
+
+
 def lq_get_device_error(device=None) -> int:
-    """Synchronizes the current stream; returns and clears the library's device error status."""
+    """Synchronizes the current stream; returns and clears the library's device error status.
+    After LQ_ERR_TIMEOUT the cached GEMM workspaces are cleared again (see _after_device_error)."""
     lib = load_library()
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     with torch.cuda.device(dev):
-        return int(lib.lq_get_device_error(_stream(dev)))
+        status = int(lib.lq_get_device_error(_stream(dev)))
+        _after_device_error(status)
+        return status
 
 
 class W4A8Linear:

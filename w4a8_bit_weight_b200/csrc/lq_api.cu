@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstdint>
 #include <cstdlib>
@@ -23,8 +24,10 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Filled once per device under g_mu; `ready` is published last (release) and
+// read first (acquire), so a thread that sees it set sees the other fields.
 struct DeviceInfo {
-  bool ready = false;
+  std::atomic<bool> ready{false};
   bool sm100 = false;
   int sms = 0;
 };
@@ -35,9 +38,9 @@ lq_status current_device(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LQ_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
+  if (!d.ready.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!d.ready) {
+    if (!d.ready.load(std::memory_order_relaxed)) {
       int major = 0, minor = 0, sms = 0;
       if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -45,7 +48,7 @@ lq_status current_device(DeviceInfo** out) {
         return LQ_ERR_CUDA;
       d.sm100 = (major == 10 && minor == 0);
       d.sms = sms;
-      d.ready = true;
+      d.ready.store(true, std::memory_order_release);
     }
   }
   *out = &d;
@@ -737,22 +740,24 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 // Device address of g_noalloc_scratch, resolved once per device.  In host code
 // the array's name only stands for the symbol; kernels must be given this
-// address.
-void* g_noalloc_addr[kMaxDevices] = {};
+// address.  The entries are atomics: a thread may read one while another
+// publishes it under the mutex (acquire load, release store).
+std::atomic<void*> g_noalloc_addr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
 lq_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LQ_ERR_CUDA;
-  if (!g_noalloc_addr[dev]) {
+  void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-      void* p = nullptr;
+    p = g_noalloc_addr[dev].load(std::memory_order_relaxed);
+    if (!p) {
       if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return LQ_ERR_CUDA;
-      g_noalloc_addr[dev] = p;
+      g_noalloc_addr[dev].store(p, std::memory_order_release);
     }
   }
-  *out = g_noalloc_addr[dev];
+  *out = p;
   return LQ_OK;
 }
 
