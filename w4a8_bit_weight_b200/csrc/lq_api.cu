@@ -89,6 +89,21 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The activations of a split-K CTA's first `stages` K-blocks as one 3D box:
+// x_q [M][K] viewed as [K/128 blocks][M tokens][128 bytes]; a box is `stages`
+// blocks x bt tokens, which is the tile kernel's shared-memory ring layout.
+bool make_map_x3(CUtensorMap* m, const void* x_q, int M, int K, int bt, int stages) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)lq::kBlockK, (cuuint64_t)M, (cuuint64_t)(K / lq::kBlockK)};
+  const cuuint64_t strides[2] = {(cuuint64_t)K, (cuuint64_t)lq::kBlockK};
+  const cuuint32_t box[3] = {(cuuint32_t)lq::kBlockK, (cuuint32_t)bt, (cuuint32_t)stages};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(x_q), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------- schedule
 enum SchedKind { kSchedAuto = 0, kSchedTiles = 1, kSchedPersistent = 2, kSchedStreamK = 3, kSchedPair = 4 };
 
@@ -306,40 +321,55 @@ lq_status launch_ex(Kern kern, int grid, int block, int smem, int cluster, bool 
   return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
 }
 
+// The tile kernel's second activation map: for cluster schedules the 3D box of
+// the first kStages K-blocks (make_map_x3), else a placeholder the kernel never
+// reads.
+template <int BT, int CS, int DQ>
+bool make_tile_x3(CUtensorMap* tx3, const CUtensorMap& tx, const void* x_q, const lq::GemmArgs& a) {
+  if constexpr (CS >= 1) {
+    return make_map_x3(tx3, x_q, a.M, a.K, BT, lq::GemmCfg<BT, CS, DQ>::kStages);
+  } else {
+    *tx3 = tx;
+    return true;
+  }
+}
+
 template <int BT, int CS, bool I32>
-lq_status launch_gemm_t(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
-                        const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+lq_status launch_gemm_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                        const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   using C = lq::GemmCfg<BT, CS>;
   auto kern = lq::w4a8_gemm_kernel<BT, CS, I32>;
+  CUtensorMap tx3;
+  if (!make_tile_x3<BT, CS, 0>(&tx3, tx, x_q, a)) return LQ_ERR_CUDA;
   // the attribute is per function and cheap; set it on every call so that any
   // device current at call time is covered
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return LQ_ERR_CUDA;
-  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tw, ts, ta, a);
+  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, ts, ta, a);
 }
 
 template <int BT, bool I32>
-lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
-                         const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                         const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   switch (s.cs) {
-    case 0: return launch_gemm_t<BT, 0, I32>(s, tx, tw, ts, ta, a, st);
-    case 1: return launch_gemm_t<BT, 1, I32>(s, tx, tw, ts, ta, a, st);
+    case 0: return launch_gemm_t<BT, 0, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 1: return launch_gemm_t<BT, 1, I32>(s, tx, x_q, tw, ts, ta, a, st);
     case 2:
-      if constexpr (BT <= 128) return launch_gemm_t<BT, 2, I32>(s, tx, tw, ts, ta, a, st);
+      if constexpr (BT <= 128) return launch_gemm_t<BT, 2, I32>(s, tx, x_q, tw, ts, ta, a, st);
       break;
     case 4:
-      if constexpr (BT <= 128) return launch_gemm_t<BT, 4, I32>(s, tx, tw, ts, ta, a, st);
+      if constexpr (BT <= 128) return launch_gemm_t<BT, 4, I32>(s, tx, x_q, tw, ts, ta, a, st);
       break;
     case 8:
-      if constexpr (BT <= 32) return launch_gemm_t<BT, 8, I32>(s, tx, tw, ts, ta, a, st);
+      if constexpr (BT <= 32) return launch_gemm_t<BT, 8, I32>(s, tx, x_q, tw, ts, ta, a, st);
       break;
   }
   return LQ_ERR_INVALID_ARG;
 }
 
 template <bool I32>
-lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
-                      const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                      const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   if (s.kind == kSchedPair) {
     auto kern = lq::w4a8_gemm_pair_kernel<I32>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::kQSmemBytes) != cudaSuccess)
@@ -353,11 +383,11 @@ lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMa
     return launch_ex(kern, s.grid, lq::kPThreads, lq::kPSmemBytes, 1, pdl_enabled(), st, tx, tw, ts, ta, a);
   }
   switch (s.bt) {
-    case 16: return launch_gemm_bt<16, I32>(s, tx, tw, ts, ta, a, st);
-    case 32: return launch_gemm_bt<32, I32>(s, tx, tw, ts, ta, a, st);
-    case 64: return launch_gemm_bt<64, I32>(s, tx, tw, ts, ta, a, st);
-    case 128: return launch_gemm_bt<128, I32>(s, tx, tw, ts, ta, a, st);
-    case 256: return launch_gemm_bt<256, I32>(s, tx, tw, ts, ta, a, st);
+    case 16: return launch_gemm_bt<16, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 32: return launch_gemm_bt<32, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 64: return launch_gemm_bt<64, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 128: return launch_gemm_bt<128, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 256: return launch_gemm_bt<256, I32>(s, tx, x_q, tw, ts, ta, a, st);
   }
   return LQ_ERR_INVALID_ARG;
 }
@@ -366,27 +396,29 @@ lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const CUtensorMa
 // kernel with per-element expansion (bit 0) and/or A expanded into shared
 // memory (bit 1), for 16- and 64-token tiles in 4-CTA clusters.
 template <int BT, int CS, bool I32, int DQ>
-lq_status launch_abl_t(const Schedule& s, const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& ts,
-                       const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+lq_status launch_abl_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                       const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   using C = lq::GemmCfg<BT, CS, DQ>;
   auto kern = lq::w4a8_gemm_kernel<BT, CS, I32, false, DQ>;
+  CUtensorMap tx3;
+  if (!make_tile_x3<BT, CS, DQ>(&tx3, tx, x_q, a)) return LQ_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return LQ_ERR_CUDA;
-  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tw, ts, ta, a);
+  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, ts, ta, a);
 }
 
 template <bool I32>
-lq_status launch_ablation(const Schedule& s, int dq, const CUtensorMap& tx, const CUtensorMap& tw,
+lq_status launch_ablation(const Schedule& s, int dq, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
                           const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
-  if (dq == 0) return launch_gemm<I32>(s, tx, tw, ts, ta, a, st);
+  if (dq == 0) return launch_gemm<I32>(s, tx, x_q, tw, ts, ta, a, st);
   if (s.kind != kSchedTiles || s.cs != 4) return LQ_ERR_UNSUPPORTED_SHAPE;
   switch (s.bt * 4 + dq) {
-    case 16 * 4 + 1: return launch_abl_t<16, 4, I32, 1>(s, tx, tw, ts, ta, a, st);
-    case 16 * 4 + 2: return launch_abl_t<16, 4, I32, 2>(s, tx, tw, ts, ta, a, st);
-    case 16 * 4 + 3: return launch_abl_t<16, 4, I32, 3>(s, tx, tw, ts, ta, a, st);
-    case 64 * 4 + 1: return launch_abl_t<64, 4, I32, 1>(s, tx, tw, ts, ta, a, st);
-    case 64 * 4 + 2: return launch_abl_t<64, 4, I32, 2>(s, tx, tw, ts, ta, a, st);
-    case 64 * 4 + 3: return launch_abl_t<64, 4, I32, 3>(s, tx, tw, ts, ta, a, st);
+    case 16 * 4 + 1: return launch_abl_t<16, 4, I32, 1>(s, tx, x_q, tw, ts, ta, a, st);
+    case 16 * 4 + 2: return launch_abl_t<16, 4, I32, 2>(s, tx, x_q, tw, ts, ta, a, st);
+    case 16 * 4 + 3: return launch_abl_t<16, 4, I32, 3>(s, tx, x_q, tw, ts, ta, a, st);
+    case 64 * 4 + 1: return launch_abl_t<64, 4, I32, 1>(s, tx, x_q, tw, ts, ta, a, st);
+    case 64 * 4 + 2: return launch_abl_t<64, 4, I32, 2>(s, tx, x_q, tw, ts, ta, a, st);
+    case 64 * 4 + 3: return launch_abl_t<64, 4, I32, 3>(s, tx, x_q, tw, ts, ta, a, st);
   }
   return LQ_ERR_UNSUPPORTED_SHAPE;
 }
@@ -445,9 +477,10 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   a.U = s.U;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (dq != 0)
-    return out_i32 ? launch_ablation<true>(s, dq, tx, tw, ts, ta, a, cs)
-                   : launch_ablation<false>(s, dq, tx, tw, ts, ta, a, cs);
-  return out_i32 ? launch_gemm<true>(s, tx, tw, ts, ta, a, cs) : launch_gemm<false>(s, tx, tw, ts, ta, a, cs);
+    return out_i32 ? launch_ablation<true>(s, dq, tx, x_q, tw, ts, ta, a, cs)
+                   : launch_ablation<false>(s, dq, tx, x_q, tw, ts, ta, a, cs);
+  return out_i32 ? launch_gemm<true>(s, tx, x_q, tw, ts, ta, a, cs)
+                 : launch_gemm<false>(s, tx, x_q, tw, ts, ta, a, cs);
 }
 
 // ---------------------------------------- fused activation quantization
@@ -479,8 +512,8 @@ lq_status launch_fused_t(const Schedule& s, const CUtensorMap& tw, const CUtenso
   auto kern = lq::w4a8_gemm_kernel<16, CS, false, true>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return LQ_ERR_CUDA;
-  // no activation tensor map: the weight map stands in for it (never used)
-  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tw, tw, ts, ta, a);
+  // no activation tensor maps: the weight map stands in for them (never used)
+  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tw, tw, tw, ts, ta, a);
 }
 
 size_t align16(size_t b) { return (b + 15) / 16 * 16; }
@@ -862,7 +895,8 @@ lq_status grouped_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, c
   a.m_off = m_off;
   a.groups = groups;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return out_i32 ? launch_gemm<true>(s, tx, tw, ts, ta, a, cs) : launch_gemm<false>(s, tx, tw, ts, ta, a, cs);
+  return out_i32 ? launch_gemm<true>(s, tx, x_q, tw, ts, ta, a, cs)
+                 : launch_gemm<false>(s, tx, x_q, tw, ts, ta, a, cs);
 }
 
 }  // namespace

@@ -94,14 +94,12 @@ struct GemmCfg {
   static constexpr int kSlots = BT <= 64 ? (kStages < (256 - kAccCols) / 32 ? kStages : (256 - kAccCols) / 32)
                                          : kStages;
   static constexpr int kTmemCols = (kAccCols + kSlots * 32 <= 256) ? 256 : 512;
-  // Cluster split-K is a reduce-scatter: the tile's 128 x BT partial sums are cut
-  // into CS pieces (row quarters, and token slices of them when CS = 8); each
-  // CTA owns one piece (CS = 2: two quarters) and receives it from the others.
-  static constexpr int kSlices = CS >= 4 ? CS / 4 : 1;            // token slices per row quarter
-  static constexpr int kPieceT = BT / kSlices;                    // tokens per piece
-  static constexpr int kOwned = CS >= 4 ? 1 : (CS == 2 ? 2 : 4);  // pieces (quarters) owned per CTA
-  static constexpr int kPieceBytes = kPieceT * 32 * 4;            // [tokens][32 rows] int32
-  static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * kOwned * kPieceBytes : 0;  // received pieces
+  // Cluster split-K is a reduce-scatter over token slices: CTA rank o owns
+  // tokens [o kT, (o + 1) kT) of the tile for all 128 weight rows; every other
+  // CTA sends it those columns of its partial sums straight from registers
+  // (st.async into [source][row][kT] int32, counted on the owner's barrier).
+  static constexpr int kT = CS >= 2 ? BT / CS : BT;                // tokens per owner
+  static constexpr int kRedBytes = CS >= 2 ? (CS - 1) * kBlockN * kT * 4 : 0;  // received slices
   static constexpr int kXRing = kStages * kXBytes;
   static constexpr int kASmem = (DQ & 2) ? kSlots * kBlockN * kBlockK : 0;  // explicit pipeline: int8 A tiles, SW128
   static constexpr int kWRing = kStages * kWStage;
@@ -117,13 +115,14 @@ struct GemmCfg {
   static_assert(kAccCols + kSlots * 32 <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kXBytes % 1024 == 0 && (kXRing + kASmem + kWRing + kRedBytes) % 8 == 0, "alignment");
-  static_assert(4 * kStages * 8 + 2 * kSlots * 8 + 8 * 8 + 16 <= 512, "barrier area");
+  static_assert((3 * kStages + 2 * kSlots + 9) * 8 + 16 <= 512, "barrier area");
   // One K-block more than TMEM slots and no refills (a 16- or 32-token decode
   // CTA holding its whole K-slice): the extra block is expanded into the
   // shared memory of weight stages 0-1 (free by then) and multiplied with A
   // from shared memory, instead of waiting for slot 0 to be released.
   static_assert(kSlots < 2 || 128 * kBlockK <= 2 * kWStage, "overflow block fits two weight stages");
   static_assert(512 + 8 * 16 * 4 + 16 * 4 <= 1088 && 1088 + 4 * 4 <= kBarBytes, "fused-quantization and progress area");
+  static_assert(CS < 2 || (kT >= 2 && kT % 2 == 0 && (kT == 2 || kT % 4 == 0)), "token slice: 2 or a multiple of 4");
 };
 
 struct GemmArgs {
@@ -299,6 +298,18 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&v)[32]
   }
 }
 
+// Reads W accumulator columns of this warp's 32 TMEM lanes and waits for them.
+template <int W>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[W]) {
+  static_assert(W == 2 || W == 4 || W == 8 || W == 16 || W == 32, "TMEM load width");
+  if constexpr (W == 2) tmem_ld_32x32b_x2(taddr, v);
+  if constexpr (W == 4) tmem_ld_32x32b_x4(taddr, v);
+  if constexpr (W == 8) tmem_ld_32x32b_x8(taddr, v);
+  if constexpr (W == 16) tmem_ld_32x32b_x16(taddr, v);
+  if constexpr (W == 32) tmem_ld_32x32b_x32(taddr, v);
+  tmem_ld_wait();
+}
+
 // CTAs that keep to 256 TMEM columns are meant to share an SM with a CTA of
 // the next launch (programmatic dependent launch): registers are capped for two.
 //
@@ -309,9 +320,9 @@ __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t (&v)[32]
 // tiles; the row maxima are combined over the cluster through DSMEM.
 template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0>
 __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols == 256 ? 2 : 1)
-    w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
-                     const GemmArgs p) {
+    w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_x3,
+                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                     const __grid_constant__ CUtensorMap tm_a, const GemmArgs p) {
   using C = GemmCfg<BT, CS, DQ>;
   static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
   static_assert(DQ == 0 || (!FQ && CS >= 1), "ablation variants: plain tile schedules only");
@@ -339,7 +350,8 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   uint64_t* xfirst = redbar + 1;  // the activation tiles of the first min(S, total) K-blocks, all at once
   uint64_t* amaxbar = xfirst + 1;  // FQ: the other CTAs' partial row maxima have landed
   uint64_t* ovfull = amaxbar + 1;  // the overflow K-block is expanded in shared memory
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ovfull + 1);
+  uint64_t* drain2 = ovfull + 1;   // the second MMA issuer's MMAs have finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain2 + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   float* amx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(wfull) + 512);  // FQ: [CS][16]
@@ -371,6 +383,38 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   auto xrow_of = [&](int tm) { return grouped ? g_xrow : tm * BT; };
   auto wrow_of = [&](int tn) { return grouped ? g_wrow : tn * kBlockN; };
 
+  // this CTA's range of units (tile x K-block)
+  const int KB = p.KB;
+  long long u_begin, u_end;
+  const long long U = p.U;
+  const long long G = gridDim.x;
+  if constexpr (CS >= 1) {
+    const long long t = blockIdx.x / CS;
+    const int r = (int)(blockIdx.x % CS);
+    u_begin = t * KB + (long long)r * KB / CS;
+    u_end = t * KB + (long long)(r + 1) * KB / CS;
+  } else {
+    u_begin = (long long)blockIdx.x * U / G;
+    u_end = ((long long)blockIdx.x + 1) * U / G;
+  }
+
+  // the overflow K-block (see GemmCfg): one tile, exactly one block more than slots, no refills
+  const bool ovf = !(DQ & 2) && CS >= 1 && A >= 2 && (int)(u_end - u_begin) == A + 1 && A + 1 <= S;
+
+  // Two MMA issuers (decode): 16-token tiles whose K-blocks each have a TMEM
+  // slot of their own (or the overflow block), so that no slot is reused and
+  // nothing is refilled.  A single thread issues small-N MMAs at one per ~60
+  // cycles; a second issuing warp overlaps with it.  The MMA warp takes the
+  // even K-blocks into accumulator columns [0, 16), the producer warp, idle
+  // once its loads are issued, the odd ones into [16, 32); the epilogue adds
+  // the two.
+  const int total_u = (int)(u_end - u_begin);
+  const bool dual = BT == 16 && CS >= 1 && (DQ & 2) == 0 && total_u >= 2 && (total_u <= A || ovf);
+  // Split-K clusters: whether this CTA's token slice holds any token of the tile
+  // (the other CTAs send it partial sums only then).
+  const int own_m0 = xrow_of((int)((u_begin / KB) % p.tiles_m));
+  const bool own_valid = CS >= 2 && (int)crank * C::kT < min(BT, g_mend - own_m0);
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&wfull[s], 1);
@@ -381,12 +425,13 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
       mbar_init(&afull[s], 4);
       mbar_init(&aempty[s], 1);
     }
-    mbar_init(accfull, 1);
+    mbar_init(accfull, dual ? 2 : 1);
     mbar_init(drain, 1);
+    mbar_init(drain2, 1);
     mbar_init(grp, 4);
     // every CTA of a split-K cluster expects its piece from each of the others
     mbar_init(redbar, 1);
-    if (CS >= 2) mbar_arrive_expect_tx(redbar, (uint32_t)C::kRedBytes);
+    if (CS >= 2) mbar_arrive_expect_tx(redbar, own_valid ? (uint32_t)C::kRedBytes : 0u);
     mbar_init(xfirst, FQ ? 4 : 1);  // FQ: the four quantizing warps
     mbar_init(amaxbar, 1);
     mbar_init(ovfull, 4);
@@ -395,7 +440,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     *last_flag = 0;
     for (int e = 0; e < 4; ++e) prog[e] = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tm_x);
+    if (!FQ) tma_prefetch_desc(CS >= 1 ? &tm_x3 : &tm_x);
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_s);
     tma_prefetch_desc(&tm_a);
@@ -417,27 +462,56 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   if constexpr (CS >= 2) cluster_arrive();
   bool cl_waited = false;
 
-  // this CTA's range of units (tile x K-block)
-  const int KB = p.KB;
-  long long u_begin, u_end;
-  const long long U = p.U;
-  const long long G = gridDim.x;
-  if constexpr (CS >= 1) {
-    const long long t = blockIdx.x / CS;
-    const int r = (int)(blockIdx.x % CS);
-    u_begin = t * KB + (long long)r * KB / CS;
-    u_end = t * KB + (long long)(r + 1) * KB / CS;
-  } else {
-    u_begin = (long long)blockIdx.x * U / G;
-    u_end = ((long long)blockIdx.x + 1) * U / G;
-  }
-
-  // the overflow K-block (see GemmCfg): one tile, exactly one block more than slots, no refills
-  const bool ovf = !(DQ & 2) && CS >= 1 && A >= 2 && (int)(u_end - u_begin) == A + 1 && A + 1 <= S;
 
   // Producer and MMA warps run their loops with all 32 lanes (one lane issues),
   // so every warp stays converged up to the CTA barrier at teardown.
   const bool leader = (lane == 0);
+
+  // The dual-issue form of the MMA loop (see `dual`): issuer i takes the
+  // K-blocks b = i, i + 2, ... into accumulator columns [16 i, 16 i + 16).
+  // Expansion finishes K-blocks in order, so a completed last block covers
+  // every block before it; each slot is used once (phase 0).  Returns whether
+  // this issuer has MMAs in flight (to be drained before TMEM is freed).
+  auto dual_issue = [&](int i) -> bool {
+    bool ok = true;
+    if (leader) {
+      constexpr uint32_t idesc = idesc_i8(BT);
+      ok = mbar_wait(xfirst, 0, abort_flag);
+      const int bl = ((total_u - 1 - i) & 1) ? total_u - 2 : total_u - 1;  // last block of this issuer
+      if (ok && !(ovf && bl == A ? mbar_try_wait(smem_u32(ovfull), 0) : mbar_try_wait(smem_u32(&afull[bl]), 0)))
+        for (int b = i; b <= bl && ok; b += 2)
+          ok = (ovf && b == A) ? mbar_wait(ovfull, 0, abort_flag) : mbar_wait(&afull[b], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(16 * i);
+        for (int b = i; b < total_u; b += 2) {
+          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + b * C::kXBytes));
+          if (ovf && b == A) {
+            // the overflow block: A from the weight stages it was expanded into
+            const uint64_t adesc = smem_desc_k_sw128(smem_u32(wring));
+#pragma unroll
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_i8_ss(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+          } else {
+            const uint32_t a_col = tmem_base + C::kAccCols + b * 32;
+#pragma unroll
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_i8_ts(d, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(accfull);
+      }
+    }
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  };
+  // waits (bounded) until this thread's issued MMAs have finished
+  auto drain_mmas = [&](uint64_t* bar) {
+    tc_commit(bar);
+    const uint32_t a = smem_u32(bar);
+    const unsigned long long t0w = globaltimer();
+    while (!mbar_try_wait(a, 0) && globaltimer() - t0w < 100000000ull) {
+    }
+  };
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Weight tiles depend on nothing the preceding kernel writes: the first
@@ -467,10 +541,19 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     griddep_wait();
     if (leader && P > 0 && !FQ) {
       // one barrier for all of them: the MMA warp waits once
-      mbar_arrive_expect_tx(xfirst, (uint32_t)P * C::kTxX);
-      UnitCursor cx = first;
-      for (int i = 0; i < P; ++i, cx.next(KB, p.tiles_m))
-        tma_load_2d(xring + i * C::kXBytes, &tm_x, xfirst, cx.kb * kBlockK, xrow_of(cx.tile_m), pol_keep);
+      if constexpr (CS >= 1) {
+        // a cluster CTA's K-blocks are consecutive blocks of one tile: the first
+        // S of them in one 3D box [block][token][128 bytes], which is the ring's
+        // layout (blocks past the CTA's slice are loaded and not used; blocks
+        // past K read as zero)
+        mbar_arrive_expect_tx(xfirst, (uint32_t)S * C::kTxX);
+        tma_load_3d(xring, &tm_x3, xfirst, 0, xrow_of(first.tile_m), first.kb, pol_keep);
+      } else {
+        mbar_arrive_expect_tx(xfirst, (uint32_t)P * C::kTxX);
+        UnitCursor cx = first;
+        for (int i = 0; i < P; ++i, cx.next(KB, p.tiles_m))
+          tma_load_2d(xring + i * C::kXBytes, &tm_x, xfirst, cx.kb * kBlockK, xrow_of(cx.tile_m), pol_keep);
+      }
     }
     __syncwarp();
     // xfull[s] serves the refills of stage s only: its k-th phase is the (k+1)-th use of the stage
@@ -517,6 +600,10 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
           }
       }
     }
+    if (dual && dual_issue(1) && leader) drain_mmas(drain2);
+  } else if (warp == 1 && dual) {
+    // ------------------------------------------- MMA issuer (dual form)
+    if (dual_issue(0) && leader) drain_mmas(drain);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = idesc_i8(BT);
@@ -865,47 +952,30 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
       const int mend = g_mend;             // rows from here on are not this tile's
       const bool n_ok = n < p.N;
       const float sc = (!OUT_I32 && n_ok) ? __ldg(p.s_c + g_scoff + n) : 0.0f;
-      // the first token this warp writes: split-K clusters write only their own piece
-      constexpr int SXC = CS >= 2 ? (C::kPieceT < 32 ? C::kPieceT : 32) : CH;
-      const int sx0 = m0 + (CS >= 4 ? (int)(crank % C::kSlices) * C::kPieceT : 0);
+      // token scales, lane-distributed (token i of the chunk: lane i): direct
+      // epilogues take the tile's tokens from m0, split-K clusters this CTA's
+      // token slice from m0 + crank kT (registers j: tokens 32 j + lane)
+      constexpr int SXC = CS >= 2 ? (C::kT < 32 ? C::kT : 32) : CH;
+      constexpr int kSxRegs = CS >= 2 ? (C::kT + 31) / 32 : 1;
+      const int sx0 = m0 + (CS >= 2 ? (int)crank * C::kT : 0);
       float sx_next = 0.0f;
+      float sxr[kSxRegs];
+#pragma unroll
+      for (int j = 0; j < kSxRegs; ++j) sxr[j] = 0.0f;
       if constexpr (FQ) {
         // s_x from the quantizing warps (all four have arrived on xfirst)
         if (!__all_sync(0xffffffffu, mbar_wait(xfirst, 0, abort_flag))) goto epi_done;
-        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? sxs[sx0 - m0 + lane] : 0.0f;
-      } else {
-        sx_next = (!OUT_I32 && lane < SXC && sx0 + lane < mend) ? ld_dep(p.s_x + sx0 + lane) : 0.0f;
       }
-      // split-K clusters: the scales of the piece this thread will write (the
-      // reduce-scatter's owner phase), also loaded before the accumulator wait.
-      // In that phase lane l takes rows 4 (l % 8) .. 4 (l % 8) + 3 of the owned
-      // quarter (16-byte reads of the staged partial sums) and token l / 8 of
-      // each group of four of the warp's tokens.
-      constexpr int kWarpsPerPiece = 4 / C::kOwned;         // CS = 2: two quarters, two warps each
-      constexpr int kTok = C::kPieceT / kWarpsPerPiece;     // tokens per warp in the owner phase
-      constexpr int kSxRegs = (kTok + 31) / 32;             // token i's scale: register i / 32 of lane i % 32
-      const int oe = warp - 2;
-      const int opidx = CS >= 4 ? 0 : oe % C::kOwned;
-      const int oqq = CS >= 4 ? (int)crank / C::kSlices : (int)crank * C::kOwned + opidx;  // owned quarter
-      const int ohh = CS >= 4 ? (int)crank % C::kSlices : 0;                               // owned token slice
-      const int ot0 = CS >= 4 ? oe : oe / C::kOwned;
-      const int orow = oqq * 32 + (lane & 7) * 4;           // this lane's first row in the tile
-      const int onn = tile_n * kBlockN + orow;
-      const bool onn_ok = onn < p.N;                        // N % 16 == 0: all four rows or none
-      float osc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      float osl[kSxRegs];
+      if constexpr (!OUT_I32) {
+        auto sx_at = [&](int m) { return FQ ? sxs[m - m0] : ld_dep(p.s_x + m); };
+        if constexpr (CS >= 2) {
 #pragma unroll
-      for (int j = 0; j < kSxRegs; ++j) osl[j] = 0.0f;
-      if constexpr (CS >= 2 && !OUT_I32) {
-        if (onn_ok) {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) osc[q4] = __ldg(p.s_c + g_scoff + onn + q4);
-        }
-#pragma unroll
-        for (int j = 0; j < kSxRegs; ++j) {
-          const int i = j * 32 + lane;
-          const int m = m0 + ohh * C::kPieceT + ot0 + i * kWarpsPerPiece;
-          osl[j] = (i < kTok && m < mend) ? (FQ ? sxs[m - m0] : ld_dep(p.s_x + m)) : 0.0f;
+          for (int j = 0; j < kSxRegs; ++j) {
+            const int i = 32 * j + lane;
+            sxr[j] = (i < C::kT && sx0 + i < mend) ? sx_at(sx0 + i) : 0.0f;
+          }
+        } else {
+          sx_next = (lane < SXC && sx0 + lane < mend) ? sx_at(sx0 + lane) : 0.0f;
         }
       }
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, acc_phase, abort_flag))) goto epi_done;
@@ -914,116 +984,124 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
       {
         const bool whole = (kb0 == 0 && kb1 == KB);
         if constexpr (CS >= 2) {
-          // ------------------------------ cluster split-K: reduce-scatter (DSMEM)
-          constexpr int T = C::kPieceT;
-          constexpr int TC = T < 32 ? T : 32;  // TMEM columns per load
-          const int q = sub;                   // this warp's row quarter
+          // ------------------- cluster split-K: reduce-scatter over token slices
+          // 1. the other CTAs' slices of this thread's row go straight from TMEM
+          //    to their shared memory (st.async, counted on their redbar);
+          // 2. this CTA's slice: its own partial sums plus the received ones,
+          //    scaled and stored.
+          constexpr int T = C::kT;
+          constexpr int TCH = T < 32 ? T : 32;  // TMEM columns per load
+          const int mvalid = min(BT, mend - m0);
           // the other CTAs' barriers are initialized once the whole cluster has arrived
           if (!cl_waited) {
             cluster_wait();
             cl_waited = true;
           }
-          // 1. this warp's quarter of the partial sums: TMEM -> staging rows
-          //    [token][lane] in the free activation ring
-          uint32_t* stg = reinterpret_cast<uint32_t*>(xring) + (size_t)q * BT * 32;
-#pragma unroll 1
-          for (int c = 0; c < BT / TC; ++c) {
-            uint32_t v[32];
-            const uint32_t col = (uint32_t)(c * TC);
-            if constexpr (TC == 8) {
-              uint32_t v8[8];
-              tmem_ld_32x32b_x8(t_lane + col, v8);
+          // Slice layout [source slot][row][T] int32; its 16-byte chunks are
+          // rotated by the row (chunk q at q ^ (row mod T/4)) so that the
+          // owner's 16-byte reads of consecutive rows fall in different banks.
+          auto red_off = [&](int slot, int q4) -> int {  // int32 offset of chunk q4 (4 values) of row r
+            constexpr int kC = T / 4;
+            const int q = kC >= 2 ? (q4 ^ (r & (kC - 1))) : q4;
+            return (slot * kBlockN + r) * T + 4 * q;
+          };
+          auto send = [&](int o, int c0, const uint32_t* v) {  // columns [c0, c0 + TCH) of slice o
+            const int slot = (int)crank < o ? (int)crank : (int)crank - 1;
+            const uint32_t bar = mapa_shared(smem_u32(redbar), (uint32_t)o);
+            if constexpr (T == 2) {
+              st_async_v2(mapa_shared(smem_u32(red + (slot * kBlockN + r) * 2), (uint32_t)o), v[0], v[1], bar);
+            } else {
+#pragma unroll
+              for (int q = 0; q < TCH; q += 4)
+                st_async_v4(mapa_shared(smem_u32(red + red_off(slot, (c0 + q) / 4)), (uint32_t)o), v[q], v[q + 1],
+                            v[q + 2], v[q + 3], bar);
+            }
+          };
+          uint32_t own16[BT == 16 ? T : 1];  // 16-token tiles: this CTA's slice, kept from the one load
+          if constexpr (BT == 16) {
+            uint32_t v[16];
+            if (dual) {
+              uint32_t w[32];
+              tmem_ld_32x32b_x32(t_lane, w);
               tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = v8[i];
+              for (int i = 0; i < 16; ++i) v[i] = w[i] + w[16 + i];
             } else {
-              tmem_load_cols<TC>(t_lane + col, v);
+              tmem_ld_32x32b_x16(t_lane, v);
+              tmem_ld_wait();
             }
 #pragma unroll
-            for (int i = 0; i < TC; ++i) stg[(col + i) * 32 + lane] = v[i];
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          // 2. the pieces other CTAs own: one bulk copy each, counted on the owner's barrier
-          bool sent = false;
-#pragma unroll 1
-          for (int h = 0; h < C::kSlices; ++h) {
-            const int o = CS >= 4 ? q * C::kSlices + h : q / C::kOwned;
-            if (o == (int)crank) continue;
-            if (lane == 0) {
-              const int slot = (int)crank < o ? (int)crank : (int)crank - 1;
-              const int pidx = CS >= 4 ? 0 : q % C::kOwned;
-              const uint32_t dst = mapa_shared(smem_u32(red + ((size_t)slot * C::kOwned + pidx) * T * 32), (uint32_t)o);
-              bulk_copy_s2s(dst, stg + (size_t)h * T * 32, (uint32_t)C::kPieceBytes, mapa_shared(smem_u32(redbar), (uint32_t)o));
-              bulk_commit();
+            for (int o = 0; o < CS; ++o) {
+              if (o == (int)crank) {
+#pragma unroll
+                for (int i = 0; i < T; ++i) own16[i] = v[o * T + i];
+              } else if (o * T < mvalid) {
+                send(o, 0, v + o * T);
+              }
             }
-            sent = true;
+          } else {
+#pragma unroll
+            for (int o = 0; o < CS; ++o) {
+              if (o == (int)crank || o * T >= mvalid) continue;
+#pragma unroll 1
+              for (int c0 = 0; c0 < T; c0 += TCH) {
+                uint32_t v[TCH];
+                tmem_ld_cols<TCH>(t_lane + (uint32_t)(o * T + c0), v);
+                send(o, c0, v);
+              }
+            }
           }
-          // 3. this CTA's own piece, shared by all four warps: the owning
-          //    warp's staged partial (visible after the group barrier) plus
-          //    the others' pieces (visible after their bytes have landed)
-          if (!group_sync(grp, grp_phase, abort_flag)) goto epi_done;
-          // every lane observes the completed bytes itself (cluster-scope acquire)
-          if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
+          if (own_valid) {
+            // every lane observes the completed bytes itself (cluster-scope acquire)
+            if (!__all_sync(0xffffffffu, mbar_wait_cluster(redbar, 0, abort_flag))) goto epi_done;
+          }
           red_done = true;
-          {
-            const uint32_t* own = reinterpret_cast<const uint32_t*>(xring) + (size_t)oqq * BT * 32 + (size_t)ohh * T * 32;
-            const uint32_t* rsrc = reinterpret_cast<const uint32_t*>(red) + (size_t)opidx * T * 32;
-            const int tsub = lane >> 3;  // token of the group of four
-            const int rcol = (lane & 7) * 4;
-            // two groups (8 tokens) per step: all their partial sums are read
-            // before any of their stores (a store may not be moved above a
-            // later load of shared memory the compiler cannot tell apart from it)
-            constexpr int kGroups = (kTok + 3) / 4;
-            constexpr int kGC = kGroups < 2 ? kGroups : 2;
+          if (own_valid) {
 #pragma unroll 1
-            for (int g0 = 0; g0 < kGroups; g0 += kGC) {
-              uint4 acc[kGC];
-              int tk[kGC];
+            for (int c0 = 0; c0 < T; c0 += TCH) {
+              uint32_t acc[TCH];
+              if constexpr (BT == 16) {
 #pragma unroll
-              for (int c = 0; c < kGC; ++c) {
-                const int i = (g0 + c) * 4 + tsub;  // this lane's token among the warp's
-                tk[c] = ot0 + (i < kTok ? i : 0) * kWarpsPerPiece;  // token within the piece
-                acc[c] = *reinterpret_cast<const uint4*>(own + tk[c] * 32 + rcol);
-#pragma unroll
-                for (int sidx = 0; sidx < CS - 1; ++sidx) {
-                  const uint4 v = *reinterpret_cast<const uint4*>(rsrc + (size_t)sidx * C::kOwned * T * 32 + tk[c] * 32 + rcol);
-                  acc[c].x += v.x;
-                  acc[c].y += v.y;
-                  acc[c].z += v.z;
-                  acc[c].w += v.w;
-                }
+                for (int i = 0; i < TCH; ++i) acc[i] = own16[i];
+              } else {
+                tmem_ld_cols<TCH>(t_lane + (uint32_t)((int)crank * T + c0), acc);
               }
 #pragma unroll
-              for (int c = 0; c < kGC; ++c) {
-                const int i = (g0 + c) * 4 + tsub;
-                const int m = m0 + ohh * T + tk[c];
-                // the token's scale, already in registers (lane-distributed)
-                float sxm = 0.0f;
-                if constexpr (!OUT_I32)
-                  sxm = __shfl_sync(0xffffffffu, (kSxRegs == 1 || (g0 + c) * 4 < 32) ? osl[0] : osl[kSxRegs - 1], i & 31);
-                if (i < kTok && m < mend && onn_ok) {
-                  if constexpr (OUT_I32) {
-                    *reinterpret_cast<uint4*>(reinterpret_cast<int32_t*>(p.out) + (size_t)m * p.N + onn) = acc[c];
-                  } else {
-                    const uint32_t av[4] = {acc[c].x, acc[c].y, acc[c].z, acc[c].w};
-                    uint32_t h[2];
+              for (int sidx = 0; sidx < CS - 1; ++sidx) {
+                if constexpr (T == 2) {
+                  const uint2 w2 = *reinterpret_cast<const uint2*>(red + (sidx * kBlockN + r) * 2);
+                  acc[0] += w2.x;
+                  acc[1] += w2.y;
+                } else {
 #pragma unroll
-                    for (int q2 = 0; q2 < 2; ++q2) {
-                      const float y0 = __fmul_rn(__int2float_rn((int32_t)av[2 * q2]), __fmul_rn(sxm, osc[2 * q2]));
-                      const float y1 = __fmul_rn(__int2float_rn((int32_t)av[2 * q2 + 1]), __fmul_rn(sxm, osc[2 * q2 + 1]));
-                      const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-                      h[q2] = *reinterpret_cast<const uint32_t*>(&b2);
-                    }
-                    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.N + onn) = make_uint2(h[0], h[1]);
+                  for (int q = 0; q < TCH; q += 4) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(red + red_off(sidx, (c0 + q) / 4));
+                    acc[q] += w4.x;
+                    acc[q + 1] += w4.y;
+                    acc[q + 2] += w4.z;
+                    acc[q + 3] += w4.w;
+                  }
+                }
+              }
+              const float sx_chunk = (kSxRegs > 1 && c0 >= 32) ? sxr[kSxRegs - 1] : sxr[0];  // tokens c0 .. c0 + 31
+#pragma unroll
+              for (int i = 0; i < TCH; ++i) {
+                const int ti = c0 + i;  // token of the slice
+                const int m = sx0 + ti;
+                float sxm = 0.0f;
+                if constexpr (!OUT_I32) sxm = __shfl_sync(0xffffffffu, sx_chunk, i);
+                if (m < mend && n_ok) {
+                  if constexpr (OUT_I32) {
+                    reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)acc[i];
+                  } else {
+                    const float y = __fmul_rn(__int2float_rn((int32_t)acc[i]), __fmul_rn(sxm, sc));
+                    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
                   }
                 }
               }
             }
           }
           tc_fence_before();
-          // the staging rows are read by the bulk copies before this CTA may leave
-          if (sent && lane == 0) bulk_wait_read();
         } else {
           int32_t* ws_tile = p.ws + (size_t)t * BT * kBlockN;
 #pragma unroll 1
@@ -1032,7 +1110,15 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
             if (cc + 1 < BT / CH)
               sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < mend) ? ld_dep(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
             uint32_t v[32];
-            tmem_load_cols<CH>(t_lane + cc * CH, v);
+            if (dual) {
+              // 16-token tile, two issuers: the sum of accumulator columns [0, 16) and [16, 32)
+              tmem_ld_32x32b_x32(t_lane, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] += v[16 + i];
+            } else {
+              tmem_load_cols<CH>(t_lane + cc * CH, v);
+            }
             if (whole) {
               store_chunk<OUT_I32, CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
             } else {
@@ -1080,10 +1166,8 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
       u += kb1 - kb0;
     }
   epi_done:
-    // no bulk copy may still be reading this CTA's staging rows when it leaves
-    if (CS >= 2 && lane == 0) bulk_wait_read();
     if (!red_done) {
-      // owner on an error path: the other CTAs may still be copying into this
+      // owner on an error path: the other CTAs may still be writing into this
       // CTA's shared memory; wait (bounded) for their bytes before leaving
       const uint32_t a = smem_u32(redbar);
       const unsigned long long t0w = globaltimer();
