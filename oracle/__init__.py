@@ -248,23 +248,21 @@ def w4a8_gemm_sampled(x_q, s_x, qw, s_u8, a_u8, s_c, m_idx, n_idx, group: int = 
 def w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N: int, group: int = GROUP):
     """Grouped GEMM (one weight matrix per group, e.g. the experts of a
     mixture-of-experts layer): token rows [m_off[e], m_off[e+1]) of x_q times
-    weight rows [e*N, (e+1)*N) of the stacked quantized weights: the stacked
-    matrix is dequantized once (its packed bytes are tile-major, so a group's
-    rows are taken after the expansion), then each group is the integer GEMM
-    and the epilogue of its own rows and columns.
-    Returns (out uint16 [M,N], acc int32 [M,N])."""
+    weight rows [e*N, (e+1)*N) of the stacked quantized weights, written out
+    as one w4a8_gemm per group.  Returns (out uint16 [M,N], acc int32 [M,N])."""
     x_q = np.ascontiguousarray(x_q, np.int8)
     m_off = [int(v) for v in m_off]
     M, K = x_q.shape
-    w_hat = dequant(qw, s_u8, a_u8, group)      # [groups * N, K]
     out = np.zeros((M, N), np.uint16)
     acc = np.zeros((M, N), np.int32)
     for e in range(len(m_off) - 1):
         r0, r1 = m_off[e], m_off[e + 1]
         if r1 <= r0:
             continue
-        a = gemm_i32(x_q[r0:r1], w_hat[e * N:(e + 1) * N])
-        out[r0:r1] = epilogue(a, np.asarray(s_x)[r0:r1], np.asarray(s_c)[e * N:(e + 1) * N])
+        o, a = w4a8_gemm(x_q[r0:r1], np.asarray(s_x)[r0:r1], np.asarray(qw)[e * N:(e + 1) * N],
+                         np.asarray(s_u8)[:, e * N:(e + 1) * N], np.asarray(a_u8)[:, e * N:(e + 1) * N],
+                         np.asarray(s_c)[e * N:(e + 1) * N], group)
+        out[r0:r1] = o
         acc[r0:r1] = a
     return out, acc
 

@@ -123,37 +123,16 @@ int lq_oracle_quantize_channels(const uint16_t* W, int N, int K, int8_t* q_i8, f
 /*   s_u8 = max(1, round(R / 15))               (= floor((2R + 15) / 30))   */
 /*   Q_u4 = min(15, round(Q_u8 / s_u8))         (= floor((2Q_u8 + s)/(2s))) */
 /*   a    = 128 + mn                                                         */
-/* Packed layout (this library's own format; the review page names a       */
-/* "dual-MMA packed layout" but does not give it).  qw holds N*K/2 bytes,   */
-/* tile-major so that one 128-row x 128-K weight block is one contiguous    */
-/* run of bytes:                                                            */
-/*   rows in tiles of 128: tile t = n / 128 has R = min(128, N - 128 t)     */
-/*   rows and starts at byte 128 t (K/2);                                   */
-/*   in a tile, K in blocks of 128: block b starts at b R 64;               */
-/*   in a block, K in chunks of 32: chunk c starts at c R 16;               */
-/*   in a chunk, row r (= n mod 128) has 16 bytes at r 16: its 32 codes,    */
-/*   the little-endian 32-bit word j holding codes 8j..8j+7 of the chunk    */
-/*   with byte i (0..3) = Q_u4[8j+i] | Q_u4[8j+4+i] << 4.                   */
-/* (A last block of fewer than 128 K has fewer chunks; the offsets above    */
-/* hold unchanged.)  s_u8 and a_u8 are stored [K/G][N], N contiguous.       */
+/* Packed layout (this library's own format): row n of qw has K/2 bytes;    */
+/* the 32-bit little-endian word j of a row holds codes k = 8j..8j+7, with  */
+/* byte b (0..3) = Q_u4[8j+b] | Q_u4[8j+4+b] << 4.  s_u8 and a_u8 are       */
+/* stored [K/G][N], N contiguous.                                           */
 /* ---------------------------------------------------------------------- */
-/* Byte of qw holding code (n, k) of an N x K matrix, and which nibble. */
-static size_t packed_byte(int n, int k, int N, int K, int* high) {
-  const int t = n / 128, r = n % 128;
-  const int R = (N - 128 * t) < 128 ? (N - 128 * t) : 128;
-  const int b = k / 128, c = (k % 128) / 32, kk = k % 32;
-  const int j = kk / 8, i = (kk % 8) % 4;
-  *high = (kk % 8) >= 4;
-  return (size_t)128 * t * (size_t)(K / 2) + (size_t)b * R * 64 + (size_t)c * R * 16 + (size_t)r * 16 +
-         (size_t)(4 * j + i);
-}
-
 int lq_oracle_quantize_groups(const int8_t* q_i8, int N, int K, int G, uint8_t* qw, uint8_t* s_u8,
                               uint8_t* a_u8) {
-  if (!q_i8 || !qw || !s_u8 || !a_u8 || N < 0 || K < 0 || G <= 0 || K % G != 0 || K % 32 != 0)
+  if (!q_i8 || !qw || !s_u8 || !a_u8 || N < 0 || K < 0 || G <= 0 || K % G != 0 || K % 8 != 0)
     return ORC_ERR_ARG;
   int ngroups = K / G;
-  memset(qw, 0, (size_t)N * (K / 2));
   uint8_t* codes = (uint8_t*)malloc((size_t)K);
   if (!codes) return ORC_ERR_ARG;
   for (int n = 0; n < N; ++n) {
@@ -178,11 +157,10 @@ int lq_oracle_quantize_groups(const int8_t* q_i8, int N, int K, int G, uint8_t* 
       s_u8[(size_t)g * N + n] = (uint8_t)s;
       a_u8[(size_t)g * N + n] = (uint8_t)a;
     }
-    for (int k = 0; k < K; ++k) {
-      int high;
-      const size_t at = packed_byte(n, k, N, K, &high);
-      qw[at] = (uint8_t)(qw[at] | (high ? codes[k] << 4 : codes[k]));
-    }
+    uint8_t* prow = qw + (size_t)n * (K / 2);
+    for (int j = 0; j < K / 8; ++j)
+      for (int b = 0; b < 4; ++b)
+        prow[4 * j + b] = (uint8_t)(codes[8 * j + b] | (codes[8 * j + 4 + b] << 4));
   }
   free(codes);
   return ORC_OK;
@@ -206,14 +184,6 @@ int lq_oracle_quantize_weights(const uint16_t* W, int N, int K, int G, uint8_t* 
 /*   v = Q_u4 * s_u8 + a    (must stay in [0,255]: the UINT8 range proof)   */
 /*   Q_i8_hat = int8(v XOR 0x80)                                            */
 /* ---------------------------------------------------------------------- */
-static int unpack_tiled(const uint8_t* qw, int n, int k, int N, int K) {
-  int high;
-  const uint8_t byte = qw[packed_byte(n, k, N, K, &high)];
-  return high ? (byte >> 4) : (byte & 0x0F);
-}
-
-/* Row-major nibble order of the W4 x FP8 weights (row n has K/2 bytes; word
- * j holds codes 8j..8j+7, byte i = code[8j+i] | code[8j+4+i] << 4). */
 static int unpack_code(const uint8_t* prow, int k) {
   int j = k / 8, r = k % 8;
   uint8_t byte = prow[4 * j + (r & 3)];
@@ -229,12 +199,13 @@ static int dequant_one(int q, int s, int a, int8_t* out) {
 
 int lq_oracle_dequant(const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8, int N, int K, int G,
                       int8_t* w_i8) {
-  if (!qw || !s_u8 || !a_u8 || !w_i8 || N < 0 || K < 0 || G <= 0 || K % G != 0 || K % 32 != 0)
+  if (!qw || !s_u8 || !a_u8 || !w_i8 || N < 0 || K < 0 || G <= 0 || K % G != 0 || K % 8 != 0)
     return ORC_ERR_ARG;
   for (int n = 0; n < N; ++n) {
+    const uint8_t* prow = qw + (size_t)n * (K / 2);
     for (int k = 0; k < K; ++k) {
       int g = k / G;
-      int rc = dequant_one(unpack_tiled(qw, n, k, N, K), s_u8[(size_t)g * N + n], a_u8[(size_t)g * N + n],
+      int rc = dequant_one(unpack_code(prow, k), s_u8[(size_t)g * N + n], a_u8[(size_t)g * N + n],
                            &w_i8[(size_t)n * K + k]);
       if (rc) return rc;
     }
@@ -336,7 +307,7 @@ int lq_oracle_w4a8_gemm_sampled(const int8_t* x_q, const float* s_x, const uint8
                                 int N, int K, int G, const int64_t* m_idx, const int64_t* n_idx,
                                 int64_t count, uint16_t* out, int32_t* acc_out) {
   if (!x_q || !s_x || !qw || !s_u8 || !a_u8 || !s_c || !m_idx || !n_idx || !out || G <= 0 ||
-      K % G != 0 || K % 32 != 0)
+      K % G != 0 || K % 8 != 0)
     return ORC_ERR_ARG;
   int bad = 0;
 #pragma omp parallel for schedule(dynamic, 16) reduction(| : bad)
@@ -346,12 +317,13 @@ int lq_oracle_w4a8_gemm_sampled(const int8_t* x_q, const float* s_x, const uint8
       bad |= 1;
       continue;
     }
+    const uint8_t* prow = qw + (size_t)n * (K / 2);
     const int8_t* xr = x_q + (size_t)m * K;
     int64_t s = 0;
     for (int k = 0; k < K; ++k) {
       int g = k / G;
       int8_t w;
-      if (dequant_one(unpack_tiled(qw, (int)n, k, N, K), s_u8[(size_t)g * N + n], a_u8[(size_t)g * N + n], &w)) {
+      if (dequant_one(unpack_code(prow, k), s_u8[(size_t)g * N + n], a_u8[(size_t)g * N + n], &w)) {
         bad |= 2;
         break;
       }
