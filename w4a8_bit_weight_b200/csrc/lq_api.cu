@@ -334,18 +334,30 @@ bool make_tile_x3(CUtensorMap* tx3, const CUtensorMap& tx, const void* x_q, cons
   }
 }
 
-template <int BT, int CS, bool I32>
-lq_status launch_gemm_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
-                        const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+template <int BT, int CS, bool I32, int EG>
+lq_status launch_gemm_tg(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                         const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   using C = lq::GemmCfg<BT, CS>;
-  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32>;
+  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32, false, 0, EG>;
   CUtensorMap tx3;
   if (!make_tile_x3<BT, CS, 0>(&tx3, tx, x_q, a)) return LQ_ERR_CUDA;
   // the attribute is per function and cheap; set it on every call so that any
   // device current at call time is covered
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return LQ_ERR_CUDA;
-  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, ts, ta, a);
+  return launch_ex(kern, s.grid, lq::gemm_threads(EG), C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, ts, ta, a);
+}
+
+// Two expansion groups for 16-token cluster tiles whose CTAs preload every
+// K-block of their slice (see gemm_threads in lq_gemm_kernel.cuh).
+template <int BT, int CS, bool I32>
+lq_status launch_gemm_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                        const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  if constexpr (BT == 16 && CS >= 1) {
+    if ((s.KB + CS - 1) / CS <= lq::GemmCfg<BT, CS>::kStages)
+      return launch_gemm_tg<BT, CS, I32, 2>(s, tx, x_q, tw, ts, ta, a, st);
+  }
+  return launch_gemm_tg<BT, CS, I32, 1>(s, tx, x_q, tw, ts, ta, a, st);
 }
 
 template <int BT, bool I32>
@@ -395,16 +407,27 @@ lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const void* x_q,
 // The ablation of the dequantization pipeline (GemmCfg's DQ): the same tile
 // kernel with per-element expansion (bit 0) and/or A expanded into shared
 // memory (bit 1), for 16- and 64-token tiles in 4-CTA clusters.
-template <int BT, int CS, bool I32, int DQ>
-lq_status launch_abl_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
-                       const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+template <int BT, int CS, bool I32, int DQ, int EG>
+lq_status launch_abl_tg(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                        const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   using C = lq::GemmCfg<BT, CS, DQ>;
-  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32, false, DQ>;
+  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32, false, DQ, EG>;
   CUtensorMap tx3;
   if (!make_tile_x3<BT, CS, DQ>(&tx3, tx, x_q, a)) return LQ_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return LQ_ERR_CUDA;
-  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, ts, ta, a);
+  return launch_ex(kern, s.grid, lq::gemm_threads(EG), C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, ts, ta, a);
+}
+
+// the variants take the product kernel's expansion groups for the same shape
+template <int BT, int CS, bool I32, int DQ>
+lq_status launch_abl_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
+                       const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
+  if constexpr (BT == 16) {
+    if ((s.KB + CS - 1) / CS <= lq::GemmCfg<BT, CS, DQ>::kStages)
+      return launch_abl_tg<BT, CS, I32, DQ, 2>(s, tx, x_q, tw, ts, ta, a, st);
+  }
+  return launch_abl_tg<BT, CS, I32, DQ, 1>(s, tx, x_q, tw, ts, ta, a, st);
 }
 
 template <bool I32>
@@ -513,7 +536,7 @@ lq_status launch_fused_t(const Schedule& s, const CUtensorMap& tw, const CUtenso
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
     return LQ_ERR_CUDA;
   // no activation tensor maps: the weight map stands in for them (never used)
-  return launch_ex(kern, s.grid, lq::kGemmThreads, C::kSmemBytes, CS, pdl_enabled(), st, tw, tw, tw, ts, ta, a);
+  return launch_ex(kern, s.grid, lq::gemm_threads(1), C::kSmemBytes, CS, pdl_enabled(), st, tw, tw, tw, ts, ta, a);
 }
 
 size_t align16(size_t b) { return (b + 15) / 16 * 16; }

@@ -63,7 +63,19 @@ namespace lq {
 
 constexpr int kBlockN = 128;        // weight rows per tile (MMA M)
 constexpr int kBlockK = 128;        // K per pipeline stage (two groups of 64)
-constexpr int kGemmThreads = 192;
+// Expansion groups (template parameter EG): groups of four warps (one per
+// TMEM sub-partition) take alternate K-blocks, so that one group's TMEM
+// stores overlap the other's integer work; group 0 also runs the epilogue.
+// Two groups pay where a 16-token decode CTA expands all of its preloaded
+// K-blocks at once; where K-slices stream through the ring, the register cap
+// of ten warps costs more than the overlap gains, and they keep one.  Stream-K
+// and the fused quantization always keep one: a stream-K CTA runs several
+// tiles through one accumulator, which the epilogue must have read before the
+// next tile's first MMA (with one group the epilogue warps expanding the next
+// tile's blocks themselves imply that order); the quantizing warps need more
+// registers than two CTAs of ten warps could have.
+__host__ __device__ constexpr int gemm_threads(int eg) { return 32 * (2 + 4 * eg); }
+constexpr int kGemmThreads = gemm_threads(1);
 
 __host__ __device__ constexpr int round_up_c(int x, int a) { return (x + a - 1) / a * a; }
 __host__ __device__ constexpr int max_c(int a, int b) { return a > b ? a : b; }
@@ -105,7 +117,7 @@ struct GemmCfg {
   static constexpr int kWRing = kStages * kWStage;
   // mbarriers and flags in the first 512 bytes; with fused activation
   // quantization, the cluster's partial row maxima [CS][16] and s_x [16]
-  // after; the expansion warps' progress counters [4] at byte 1088
+  // after; the expansion warps' progress counters [4 EG] at byte 1088
   static constexpr int kBarBytes = 1152;
   static constexpr int kUsed = kXRing + kASmem + kWRing + kRedBytes + kBarBytes + 1024;  // + alignment slack
   // Shared memory also bounds how many CTAs share an SM: a 512-column CTA
@@ -121,7 +133,8 @@ struct GemmCfg {
   // shared memory of weight stages 0-1 (free by then) and multiplied with A
   // from shared memory, instead of waiting for slot 0 to be released.
   static_assert(kSlots < 2 || 128 * kBlockK <= 2 * kWStage, "overflow block fits two weight stages");
-  static_assert(512 + 8 * 16 * 4 + 16 * 4 <= 1088 && 1088 + 4 * 4 <= kBarBytes, "fused-quantization and progress area");
+  static_assert(512 + 8 * 16 * 4 + 16 * 4 <= 1088 && 1088 + 4 * 2 * 4 <= kBarBytes,
+                "fused-quantization and progress area");
   static_assert(CS < 2 || (kT >= 2 && kT % 2 == 0 && (kT == 2 || kT % 4 == 0)), "token slice: 2 or a multiple of 4");
 };
 
@@ -152,6 +165,15 @@ struct UnitCursor {
     tile_n = t / tiles_m;
     tile_m = t - tile_n * tiles_m;
   }
+  // the cursor at K-block kb of tile t (32-bit arithmetic only)
+  __device__ __forceinline__ static UnitCursor at(int t, int kb, int tiles_m) {
+    UnitCursor c;
+    c.kb = kb;
+    c.tile_n = t / tiles_m;
+    c.tile_m = t - c.tile_n * tiles_m;
+    return c;
+  }
+  UnitCursor() = default;
   __device__ __forceinline__ void next(int KB, int tiles_m) {
     if (++kb == KB) {
       kb = 0;
@@ -318,12 +340,14 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[W]) {
 // the expansion warps quantize them (per-token symmetric INT8, the same
 // arithmetic as quantize_act_kernel) straight into the swizzled activation
 // tiles; the row maxima are combined over the cluster through DSMEM.
-template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0>
-__global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols == 256 ? 2 : 1)
+template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0, int EG = 1>
+__global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCols == 256 ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_x3,
                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                      const __grid_constant__ CUtensorMap tm_a, const GemmArgs p) {
   using C = GemmCfg<BT, CS, DQ>;
+  constexpr int kEG = EG;  // expansion groups of this variant
+  static_assert(EG == 1 || (EG == 2 && !FQ && CS >= 1), "two expansion groups: cluster schedules, no fused quantization");
   static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
   static_assert(DQ == 0 || (!FQ && CS >= 1), "ablation variants: plain tile schedules only");
   constexpr int S = C::kStages;
@@ -388,14 +412,20 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   long long u_begin, u_end;
   const long long U = p.U;
   const long long G = gridDim.x;
+  // the tile and K-block of the first unit; a 64-bit division costs hundreds
+  // of cycles, so cluster schedules (one tile per CTA) use 32-bit ones only
+  int t_first, kb_first;
   if constexpr (CS >= 1) {
-    const long long t = blockIdx.x / CS;
+    t_first = (int)(blockIdx.x / CS);
     const int r = (int)(blockIdx.x % CS);
-    u_begin = t * KB + (long long)r * KB / CS;
-    u_end = t * KB + (long long)(r + 1) * KB / CS;
+    kb_first = r * KB / CS;
+    u_begin = (long long)t_first * KB + kb_first;
+    u_end = (long long)t_first * KB + (r + 1) * KB / CS;
   } else {
     u_begin = (long long)blockIdx.x * U / G;
     u_end = ((long long)blockIdx.x + 1) * U / G;
+    t_first = (int)(u_begin / KB);
+    kb_first = (int)(u_begin - (long long)t_first * KB);
   }
 
   // the overflow K-block (see GemmCfg): one tile, exactly one block more than slots, no refills
@@ -412,7 +442,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   const bool dual = BT == 16 && CS >= 1 && (DQ & 2) == 0 && total_u >= 2 && (total_u <= A || ovf);
   // Split-K clusters: whether this CTA's token slice holds any token of the tile
   // (the other CTAs send it partial sums only then).
-  const int own_m0 = xrow_of((int)((u_begin / KB) % p.tiles_m));
+  const int own_m0 = xrow_of(t_first % p.tiles_m);
   const bool own_valid = CS >= 2 && (int)crank * C::kT < min(BT, g_mend - own_m0);
 
   if (threadIdx.x == 0) {
@@ -438,7 +468,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     if (FQ) mbar_arrive_expect_tx(amaxbar, (uint32_t)(CS - 1) * 16 * 4);
     *abort_flag = 0;
     *last_flag = 0;
-    for (int e = 0; e < 4; ++e) prog[e] = 0;
+    for (int e = 0; e < 4 * kEG; ++e) prog[e] = 0;
     fence_mbar_init();
     if (!FQ) tma_prefetch_desc(CS >= 1 ? &tm_x3 : &tm_x);
     tma_prefetch_desc(&tm_w);
@@ -525,7 +555,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     }
     const int total = (int)(u_end - u_begin);
     const int P = min(S, total);
-    const UnitCursor first(u_begin, KB, p.tiles_m);
+    const UnitCursor first = UnitCursor::at(t_first, kb_first, p.tiles_m);
     UnitCursor cw = first;  // after the prefetch: the unit of K-block P (every lane steps it)
     // first P K-blocks (they may span tiles in the stream-K schedule)
     for (int i = 0; i < P; ++i, cw.next(KB, p.tiles_m)) {
@@ -619,7 +649,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     bool any = false, x_first_seen = false;
     int it = 0, ready = 0;  // K-blocks [0, ready) are known to be expanded
     for (long long u = u_begin; u < u_end;) {
-      const int kb0 = (int)(u % KB);
+      const int kb0 = u == u_begin ? kb_first : (int)(u % KB);
       const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
       for (int kb = kb0; kb < kb1;) {
         bool ok = true;
@@ -634,9 +664,15 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
             // furthest block that is likely complete, and one look at its slot
             // (whose previous block this warp has consumed: at most A - 1
             // ahead) covers every block before it.
-            const int rep_ = min(min(prog[0], prog[1]), min(prog[2], prog[3]));
+            int rep_ = prog[0];
+#pragma unroll
+            for (int e = 1; e < 4 * kEG; ++e) rep_ = min(rep_, prog[e]);
             const int hi = min(min(rep_ - 1, it + A - 1), total - 1);
-            if (hi > it && (!ovf || hi < A) && mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u)) {
+            // each group expands its blocks in order: its latest block covers
+            // its earlier ones, so one look per group (blocks hi and hi - 1)
+            if (hi > it && (!ovf || hi < A) && mbar_try_wait(smem_u32(&afull[hi % A]), (uint32_t)(hi / A) & 1u) &&
+                (kEG == 1 ||
+                 mbar_try_wait(smem_u32(&afull[(hi - 1) % A]), (uint32_t)((hi - 1) / A) & 1u))) {
               ready = hi + 1;
             } else {
               ok = (ovf && it == A) ? mbar_wait(ovfull, 0, abort_flag)
@@ -724,6 +760,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
   } else {
     // ------------------------------------------- expansion + epilogue warps
     const int sub = warp & 3;           // TMEM sub-partition this warp may access
+    const int egrp = (warp - 2) >> 2;   // expansion group: takes the K-blocks it_e with it_e % kEG == egrp
     const int r = sub * 32 + lane;      // weight row of the tile = TMEM lane
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16);
     const int sw = (r >> 1) & 3;        // 64-byte swizzle of this row's 16-byte chunks
@@ -731,7 +768,8 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     bool waited_dep = false;
     // split-K: every epilogue warp reads this CTA's piece, so each must see all
     // of it arrive before the CTA may leave (the others' bulk copies write here)
-    bool red_done = (CS < 2);
+    bool red_done = (CS < 2) || egrp != 0;  // group 0 runs the epilogue
+    bool staged = false;  // this thread issued bulk copies from the staging rows
     int stage = 0, slot = 0;
     uint32_t sphase = 0, aphase = 0;
 
@@ -745,7 +783,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     // blocks that have a slot of their own are expanded: the next block
     // waits for an MMA, and the MMAs wait for this.
     const int total_e = (int)(u_end - u_begin);
-    bool x_done = !FQ;
+    bool x_done = !FQ || egrp != 0;
     auto fused_quantize = [&]() -> bool {
       x_done = true;
       griddep_wait();  // X may be the output of the preceding kernel
@@ -754,7 +792,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
       cl_waited = true;
       const int e = warp - 2;
       const int nchunk = total_e * (kBlockK / 32);
-      const int k0 = (int)(u_begin - (u_begin / KB) * KB) * kBlockK + lane * 32;  // this lane's first K
+      const int k0 = kb_first * kBlockK + lane * 32;  // this lane's first K
       const bool has = lane < nchunk;
       // the four tokens are independent: all loads first, then the reductions
       // and divisions side by side, so that no chain waits on another
@@ -852,20 +890,32 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
     const int x_at = ovf ? total_e : min(A, total_e);
 
     for (long long u = u_begin; u < u_end;) {
-      const int t = (int)(u / KB);
-      const int kb0 = (int)(u % KB);
+      const int t = u == u_begin ? t_first : (int)(u / KB);
+      const int kb0 = u == u_begin ? kb_first : (int)(u % KB);
       const int kb1 = (int)min((long long)KB, kb0 + (u_end - u));
       const int tile_m = t % p.tiles_m, tile_n = t / p.tiles_m;
       for (int kb = kb0; kb < kb1; ++kb, ++it_e) {
         if constexpr (FQ) {
-          if (it_e == x_at && !fused_quantize()) goto epi_done;
+          if (egrp == 0 && it_e == x_at && !fused_quantize()) goto epi_done;
+        }
+        if (it_e % kEG != egrp) {  // another group's block
+          if (++stage == S) {
+            stage = 0;
+            sphase ^= 1u;
+          }
+          if (++slot == A) {
+            slot = 0;
+            aphase ^= 1u;
+          }
+          continue;
         }
         // the overflow block goes to shared memory: it needs weight stages 0-1,
-        // which every warp has finished reading once block 1 is expanded
+        // which every warp has finished reading once blocks 0 and 1 are expanded
         const bool to_smem = ovf && it_e == A;
         // warp-uniform decision: every lane waits, all continue only if all saw the phase
         if (!__all_sync(0xffffffffu, mbar_wait(&wfull[stage], sphase, abort_flag) &&
-                                         (to_smem ? mbar_wait(&afull[1], 0, abort_flag)
+                                         (to_smem ? mbar_wait(&afull[0], 0, abort_flag) &&
+                                                        mbar_wait(&afull[1], 0, abort_flag)
                                                   : mbar_wait(&aempty[slot], aphase ^ 1u, abort_flag))))
           goto epi_done;
         tc_fence_after();
@@ -918,7 +968,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
           // a refilled block's activation tile: one warp sees it land before
           // the slot is reported ready (the MMA warp waits for the slot only)
           bool x_ok = true;
-          if (warp == 2 && it_e >= P_e && lane == 0)
+          if (sub == 2 && it_e >= P_e && lane == 0)  // the group's first warp
             x_ok = mbar_wait(&xfull[stage], (uint32_t)(it_e / S - 1) & 1u, abort_flag);
           __syncwarp();
           if (lane == 0 && x_ok) {
@@ -939,6 +989,10 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
 
       if constexpr (FQ) {
         if (!x_done && !fused_quantize()) goto epi_done;
+      }
+      if (egrp != 0) {  // the other expansion groups have no epilogue
+        u += kb1 - kb0;
+        continue;
       }
       // ------------------------------------------------------- epilogue
       if (!waited_dep) {
@@ -1039,7 +1093,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
                 send(o, 0, v + o * T);
               }
             }
-          } else {
+          } else if constexpr ((CS - 1) * T <= 32) {
 #pragma unroll
             for (int o = 0; o < CS; ++o) {
               if (o == (int)crank || o * T >= mvalid) continue;
@@ -1049,6 +1103,39 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
                 tmem_ld_cols<TCH>(t_lane + (uint32_t)(o * T + c0), v);
                 send(o, c0, v);
               }
+            }
+          } else {
+            // Large slices: per-thread remote stores would be thousands of
+            // 16-byte messages, so each warp stages its 32 rows of every other
+            // owner's slice in the free activation ring ([owner][row][T], the
+            // receive layout) and sends each with one bulk copy.
+            int32_t* stg = reinterpret_cast<int32_t*>(xring);
+#pragma unroll
+            for (int o = 0; o < CS; ++o) {
+              if (o == (int)crank || o * T >= mvalid) continue;
+#pragma unroll 1
+              for (int c0 = 0; c0 < T; c0 += TCH) {
+                uint32_t v[TCH];
+                tmem_ld_cols<TCH>(t_lane + (uint32_t)(o * T + c0), v);
+#pragma unroll
+                for (int q = 0; q < TCH; q += 4)
+                  *reinterpret_cast<uint4*>(stg + o * kBlockN * T + red_off(0, (c0 + q) / 4)) =
+                      make_uint4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+#pragma unroll 1
+              for (int o = 0; o < CS; ++o) {
+                if (o == (int)crank || o * T >= mvalid) continue;
+                const int slot = (int)crank < o ? (int)crank : (int)crank - 1;
+                bulk_copy_s2s(mapa_shared(smem_u32(red + (slot * kBlockN + sub * 32) * T), (uint32_t)o),
+                              stg + (o * kBlockN + sub * 32) * T, (uint32_t)(32 * T * 4),
+                              mapa_shared(smem_u32(redbar), (uint32_t)o));
+                staged = true;
+              }
+              bulk_commit();
             }
           }
           if (own_valid) {
@@ -1101,6 +1188,8 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
               }
             }
           }
+          // the staging rows are read by the bulk copies before this CTA may leave
+          if (staged) bulk_wait_read();
           tc_fence_before();
         } else {
           int32_t* ws_tile = p.ws + (size_t)t * BT * kBlockN;
@@ -1166,6 +1255,7 @@ __global__ void __launch_bounds__(kGemmThreads, GemmCfg<BT, CS, DQ>::kTmemCols =
       u += kb1 - kb0;
     }
   epi_done:
+    if (staged) bulk_wait_read();  // no bulk copy may still read the staging rows
     if (!red_done) {
       // owner on an error path: the other CTAs may still be writing into this
       // CTA's shared memory; wait (bounded) for their bytes before leaving
