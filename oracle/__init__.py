@@ -77,6 +77,7 @@ def _load():
         "lq_oracle_quantize_act": [P, I, I, P, P],
         "lq_oracle_gemm_i32": [P, P, I, I, I, P],
         "lq_oracle_epilogue": [P, P, P, I, I, P],
+        "lq_oracle_swiglu_epilogue": [P, P, P, I, I, P],
         "lq_oracle_w4a8_gemm": [P, P, P, P, P, P, I, I, I, I, P, P],
         "lq_oracle_w4a8_gemm_sampled": [P, P, P, P, P, P, I, I, I, I, P, P, ctypes.c_int64, P, P],
         "lq_oracle_quantize_weights_w4": [P, I, I, P, P],
@@ -205,6 +206,47 @@ def epilogue(acc: np.ndarray, s_x: np.ndarray, s_c: np.ndarray) -> np.ndarray:
     out = np.empty((M, N), np.uint16)
     _check(_load().lq_oracle_epilogue(_p(acc), _p(s_x), _p(s_c), M, N, _p(out)), "epilogue")
     return out
+
+
+def swiglu_epilogue(acc: np.ndarray, s_x: np.ndarray, s_c: np.ndarray) -> np.ndarray:
+    """SwiGLU of an interleaved gate/up pair (row 2n gate, 2n+1 up): each projection
+    float(acc) * (s_x[m] * s_c[row]) in fp32, then bf16(silu(gate) * up) with
+    silu(g) = g / (1 + exp(-g)).  acc [M, 2N] int32 -> uint16 bf16 bits [M, N]."""
+    acc = np.ascontiguousarray(acc, np.int32)
+    s_x = np.ascontiguousarray(s_x, np.float32)
+    s_c = np.ascontiguousarray(s_c, np.float32)
+    M, N2 = acc.shape
+    if N2 % 2:
+        raise ValueError("the gate/up accumulators come in pairs")
+    out = np.empty((M, N2 // 2), np.uint16)
+    _check(_load().lq_oracle_swiglu_epilogue(_p(acc), _p(s_x), _p(s_c), M, N2 // 2, _p(out)), "swiglu_epilogue")
+    return out
+
+
+def w4a8_swiglu(x_q, s_x, qw, s_u8, a_u8, s_c, group: int = GROUP):
+    """Gate/up pair of a gated FFN layer from quantized operands: the W4A8 GEMM's
+    int32 accumulators against the interleaved [2N, K] weights, then the SwiGLU
+    epilogue.  Returns (out uint16 [M, N], acc int32 [M, 2N])."""
+    _, acc = w4a8_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, group)
+    return swiglu_epilogue(acc, s_x, s_c), acc
+
+
+def w4a8_swiglu_sampled(x_q, s_x, qw, s_u8, a_u8, s_c, m_idx, n_idx, group: int = GROUP):
+    """The same for single outputs (m_idx[i], n_idx[i]) of [M, N]: the gate and up
+    accumulators of each from the sampled GEMM, then the SwiGLU epilogue."""
+    m_idx = np.asarray(m_idx, np.int64)
+    n_idx = np.asarray(n_idx, np.int64)
+    mm = np.repeat(m_idx, 2)
+    nn = np.stack([2 * n_idx, 2 * n_idx + 1], axis=1).reshape(-1)
+    _, acc = w4a8_gemm_sampled(x_q, s_x, qw, s_u8, a_u8, s_c, mm, nn, group)
+    acc = acc.reshape(-1, 2)
+    s_x = np.asarray(s_x, np.float32)
+    s_c = np.asarray(s_c, np.float32)
+    out = np.empty(len(m_idx), np.uint16)
+    for i in range(len(m_idx)):  # one output row of one column pair at a time, the same C routine
+        out[i] = swiglu_epilogue(acc[i:i + 1], s_x[m_idx[i]:m_idx[i] + 1],
+                                 s_c[2 * n_idx[i]:2 * n_idx[i] + 2])[0, 0]
+    return out, acc
 
 
 def w4a8_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, group: int = GROUP):

@@ -282,6 +282,32 @@ int lq_oracle_epilogue(const int32_t* acc, const float* s_x, const float* s_c, i
   return ORC_OK;
 }
 
+/* ---------------------------------------------------------------------- */
+/* SwiGLU epilogue of a gate/up pair (the FFN layers of the LiquidGEMM      */
+/* review page's Fig. 12 caption are Llama-style gated layers; the pages    */
+/* give no formula, the reading is the common one): the two projections of  */
+/* the same input, each with the epilogue above in fp32 (not rounded to     */
+/* bf16), then silu(gate) * up rounded once to bf16, with                   */
+/*   silu(g) = g / (1 + exp(-g))    (IEEE fp32 steps, expf from libm).      */
+/* The gate/up weights are one interleaved [2N, K] matrix quantized row by  */
+/* row: row 2n is gate channel n, row 2n+1 up channel n (this library's     */
+/* layout choice).  acc is [M, 2N], out [M, N].                             */
+/* ---------------------------------------------------------------------- */
+int lq_oracle_swiglu_epilogue(const int32_t* acc, const float* s_x, const float* s_c, int M, int N,
+                              uint16_t* out) {
+  if (!acc || !s_x || !s_c || !out || M < 0 || N < 0) return ORC_ERR_ARG;
+  for (int m = 0; m < M; ++m)
+    for (int n = 0; n < N; ++n) {
+      const int32_t* row = acc + (size_t)m * 2 * N;
+      float yg = (float)row[2 * n] * (s_x[m] * s_c[2 * n]);
+      float yu = (float)row[2 * n + 1] * (s_x[m] * s_c[2 * n + 1]);
+      float e = expf(-yg);
+      float silu = yg / (1.0f + e);
+      out[(size_t)m * N + n] = f32_to_bf16_rne(silu * yu);
+    }
+  return ORC_OK;
+}
+
 /* Whole W4A8 GEMM from already-quantized operands: dequant, contraction,
  * epilogue.  acc_out may be NULL. */
 int lq_oracle_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
