@@ -225,6 +225,35 @@ LQ_API lq_status lq_w4a8_linear_ex(const void* X_bf16, const uint8_t* qw, const 
                                    void* stream);
 
 /*
+ * lq_w4a8_gemm_swiglu -- the gate/up pair of a gated FFN layer in one GEMM
+ * with a fused SwiGLU epilogue (the FFN layers of the LiquidGEMM review page's
+ * Fig. 12 caption; the pages do not write the gated FFN out, the reading is
+ * the common one):
+ *   out[m, j] = bf16( silu(y[m, 2j]) * y[m, 2j+1] ),
+ *   y[m, n]   = float(acc[m, n]) * (s_x[m] * s_c[n])   (fp32, not rounded),
+ *   silu(g)   = g / (1 + exp(-g))                        (fp32 steps).
+ * The weights are one interleaved matrix of N = 2 * (FFN width) rows, row 2j
+ * the gate channel j and row 2j + 1 the up channel j, quantized as usual by
+ * lq_quantize_weights (per row, so interleaving changes no code).  Operands,
+ * rules and workspace as lq_w4a8_gemm with this N; out_bf16 is [M, N/2]
+ * (16-byte aligned).  The schedule is lq_w4a8_gemm's automatic one, a
+ * persistent choice replaced by one cluster per tile (the SwiGLU epilogue
+ * has no persistent or stream-K form).  exp is CUDA's expf (at most 2 ulp in
+ * fp32), so an output may differ from a correctly rounded evaluation by one
+ * bf16 ulp.
+ */
+LQ_API lq_status lq_w4a8_gemm_swiglu(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                                     const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K,
+                                     int group, void* workspace, size_t workspace_bytes, void* stream);
+/* The same with the schedule chosen as in lq_w4a8_gemm_ex (test and
+ * measurement use; LQ_SCHED_STREAMK and LQ_SCHED_PERSISTENT are refused with
+ * LQ_ERR_UNSUPPORTED_SHAPE). */
+LQ_API lq_status lq_w4a8_gemm_swiglu_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw,
+                                        const uint8_t* s_u8, const uint8_t* a_u8, const float* s_c, void* out_bf16,
+                                        int M, int N, int K, int group, void* workspace, size_t workspace_bytes,
+                                        int block_t, int schedule, int split_k, int grid, void* stream);
+
+/*
  * lq_w4a8_gemm_i32 -- the contraction only: acc[m,n] as int32 [M, N] (16-byte
  * aligned), same operands, rules and workspace as lq_w4a8_gemm.
  */

@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_gemm": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, P], I),
             "lq_w4a8_gemm_ex": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, I, I, I, I, I, P], I),
             "lq_w4a8_gemm_i32": ([P, P, P, P, P, I, I, I, I, P, Z, P], I),
+            "lq_w4a8_gemm_swiglu": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, P], I),
+            "lq_w4a8_gemm_swiglu_ex": ([P, P, P, P, P, P, P, I, I, I, I, P, Z, I, I, I, I, P], I),
             "lq_dequant_weights_i8": ([P, P, P, I, I, I, P, P], I),
             "lq_get_device_error": ([P], I),
             "lq_w4a8_gemm_noalloc": ([P, P, P, P, P, P, P, I, I, I, I, P], I),
@@ -247,6 +249,37 @@ def lq_w4a8_gemm_i32(x_q, qw, s_u8, a_u8, out=None, group: int = GROUP, block_t:
     """The int32 accumulators x_q @ dequant(qw)^T -> [M, N] int32."""
     return _gemm(x_q, None, qw, s_u8, a_u8, None, out, group, block_t, split_k, grid, True, workspace_buf,
                  schedule)
+
+
+def lq_w4a8_gemm_swiglu(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP, workspace_buf=None,
+                        block_t: int = 0, split_k: int = 0, schedule: int | None = None):
+    """Gate/up pair of a gated FFN layer in one GEMM: the weights are one interleaved
+    [2F, K] matrix (row 2j gate channel j, row 2j+1 up channel j), the output
+    bf16(silu(gate) * up) -> [M, F] bf16 (lq_w4a8_gemm_swiglu in lq.h)."""
+    lib = load_library()
+    _need(x_q, torch.int8, "x_q")
+    M, K = x_q.shape
+    N = qw.shape[0]
+    _need(qw, torch.uint8, "qw", (N, K // 2))
+    _need(s_u8, torch.uint8, "s_u8", (K // group, N))
+    _need(a_u8, torch.uint8, "a_u8", (K // group, N))
+    _need(s_x, torch.float32, "s_x", (M,))
+    _need(s_c, torch.float32, "s_c", (N,))
+    if N % 2:
+        raise ValueError("the gate/up weights come in row pairs")
+    if out is None:
+        out = torch.empty(M, N // 2, dtype=torch.bfloat16, device=x_q.device)
+    _need(out, torch.bfloat16, "out", (M, N // 2))
+    with torch.cuda.device(x_q.device):
+        ws = workspace_buf
+        sch = _sched(schedule, split_k, 0)
+        if ws is None:
+            ws = workspace(lq_w4a8_gemm_workspace_size(M, N, K, block_t, split_k, 0, sch), x_q.device)
+        nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+        _check("lq_w4a8_gemm_swiglu", lib.lq_w4a8_gemm_swiglu_ex(
+            _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out), M, N, K, group,
+            _ptr(ws), nbytes, block_t, sch, split_k, 0, _stream(x_q.device)))
+    return out
 
 
 # paths of lq_w4a8_linear (LQ_LINEAR_* in lq.h)

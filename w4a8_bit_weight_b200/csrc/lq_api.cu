@@ -334,11 +334,15 @@ bool make_tile_x3(CUtensorMap* tx3, const CUtensorMap& tx, const void* x_q, cons
   }
 }
 
-template <int BT, int CS, bool I32, int EG>
+// Output modes of the GEMM launches: bf16, int32 accumulators, or the SwiGLU
+// of an interleaved gate/up pair (bf16, half the columns).
+enum OutMode { kOutBf16 = 0, kOutI32 = 1, kOutSwiglu = 2 };
+
+template <int BT, int CS, int OUT, int EG>
 lq_status launch_gemm_tg(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
                          const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   using C = lq::GemmCfg<BT, CS>;
-  auto kern = lq::w4a8_gemm_kernel<BT, CS, I32, false, 0, EG>;
+  auto kern = lq::w4a8_gemm_kernel<BT, CS, OUT == kOutI32, false, 0, EG, OUT == kOutSwiglu>;
   CUtensorMap tx3;
   if (!make_tile_x3<BT, CS, 0>(&tx3, tx, x_q, a)) return LQ_ERR_CUDA;
   // the attribute is per function and cheap; set it on every call so that any
@@ -350,56 +354,61 @@ lq_status launch_gemm_tg(const Schedule& s, const CUtensorMap& tx, const void* x
 
 // Two expansion groups for 16-token cluster tiles whose CTAs preload every
 // K-block of their slice (see gemm_threads in lq_gemm_kernel.cuh).
-template <int BT, int CS, bool I32>
+template <int BT, int CS, int OUT>
 lq_status launch_gemm_t(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
                         const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
-  if constexpr (BT == 16 && CS >= 1) {
-    if ((s.KB + CS - 1) / CS <= lq::GemmCfg<BT, CS>::kStages)
-      return launch_gemm_tg<BT, CS, I32, 2>(s, tx, x_q, tw, ts, ta, a, st);
+  if constexpr (OUT == kOutSwiglu && CS == 0) {
+    return LQ_ERR_UNSUPPORTED_SHAPE;  // the SwiGLU epilogue has no stream-K form
+  } else {
+    if constexpr (BT == 16 && CS >= 1) {
+      if ((s.KB + CS - 1) / CS <= lq::GemmCfg<BT, CS>::kStages)
+        return launch_gemm_tg<BT, CS, OUT, 2>(s, tx, x_q, tw, ts, ta, a, st);
+    }
+    return launch_gemm_tg<BT, CS, OUT, 1>(s, tx, x_q, tw, ts, ta, a, st);
   }
-  return launch_gemm_tg<BT, CS, I32, 1>(s, tx, x_q, tw, ts, ta, a, st);
 }
 
-template <int BT, bool I32>
+template <int BT, int OUT>
 lq_status launch_gemm_bt(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
                          const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   switch (s.cs) {
-    case 0: return launch_gemm_t<BT, 0, I32>(s, tx, x_q, tw, ts, ta, a, st);
-    case 1: return launch_gemm_t<BT, 1, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 0: return launch_gemm_t<BT, 0, OUT>(s, tx, x_q, tw, ts, ta, a, st);
+    case 1: return launch_gemm_t<BT, 1, OUT>(s, tx, x_q, tw, ts, ta, a, st);
     case 2:
-      if constexpr (BT <= 128) return launch_gemm_t<BT, 2, I32>(s, tx, x_q, tw, ts, ta, a, st);
+      if constexpr (BT <= 128) return launch_gemm_t<BT, 2, OUT>(s, tx, x_q, tw, ts, ta, a, st);
       break;
     case 4:
-      if constexpr (BT <= 128) return launch_gemm_t<BT, 4, I32>(s, tx, x_q, tw, ts, ta, a, st);
+      if constexpr (BT <= 128) return launch_gemm_t<BT, 4, OUT>(s, tx, x_q, tw, ts, ta, a, st);
       break;
     case 8:
-      if constexpr (BT <= 32) return launch_gemm_t<BT, 8, I32>(s, tx, x_q, tw, ts, ta, a, st);
+      if constexpr (BT <= 32) return launch_gemm_t<BT, 8, OUT>(s, tx, x_q, tw, ts, ta, a, st);
       break;
   }
   return LQ_ERR_INVALID_ARG;
 }
 
-template <bool I32>
+template <int OUT>
 lq_status launch_gemm(const Schedule& s, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
                       const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
   if (s.kind == kSchedPair) {
-    auto kern = lq::w4a8_gemm_pair_kernel<I32>;
+    auto kern = lq::w4a8_gemm_pair_kernel<OUT == kOutI32, OUT == kOutSwiglu>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::kQSmemBytes) != cudaSuccess)
       return LQ_ERR_CUDA;
     return launch_ex(kern, s.grid, lq::kQThreads, lq::kQSmemBytes, 2, pdl_enabled(), st, tx, tw, ts, ta, a);
   }
   if (s.kind == kSchedPersistent) {
-    auto kern = lq::w4a8_gemm_persistent_kernel<I32>;
+    if constexpr (OUT == kOutSwiglu) return LQ_ERR_UNSUPPORTED_SHAPE;  // callers pick tiles instead
+    auto kern = lq::w4a8_gemm_persistent_kernel<OUT == kOutI32>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::kPSmemBytes) != cudaSuccess)
       return LQ_ERR_CUDA;
     return launch_ex(kern, s.grid, lq::kPThreads, lq::kPSmemBytes, 1, pdl_enabled(), st, tx, tw, ts, ta, a);
   }
   switch (s.bt) {
-    case 16: return launch_gemm_bt<16, I32>(s, tx, x_q, tw, ts, ta, a, st);
-    case 32: return launch_gemm_bt<32, I32>(s, tx, x_q, tw, ts, ta, a, st);
-    case 64: return launch_gemm_bt<64, I32>(s, tx, x_q, tw, ts, ta, a, st);
-    case 128: return launch_gemm_bt<128, I32>(s, tx, x_q, tw, ts, ta, a, st);
-    case 256: return launch_gemm_bt<256, I32>(s, tx, x_q, tw, ts, ta, a, st);
+    case 16: return launch_gemm_bt<16, OUT>(s, tx, x_q, tw, ts, ta, a, st);
+    case 32: return launch_gemm_bt<32, OUT>(s, tx, x_q, tw, ts, ta, a, st);
+    case 64: return launch_gemm_bt<64, OUT>(s, tx, x_q, tw, ts, ta, a, st);
+    case 128: return launch_gemm_bt<128, OUT>(s, tx, x_q, tw, ts, ta, a, st);
+    case 256: return launch_gemm_bt<256, OUT>(s, tx, x_q, tw, ts, ta, a, st);
   }
   return LQ_ERR_INVALID_ARG;
 }
@@ -433,7 +442,7 @@ lq_status launch_abl_t(const Schedule& s, const CUtensorMap& tx, const void* x_q
 template <bool I32>
 lq_status launch_ablation(const Schedule& s, int dq, const CUtensorMap& tx, const void* x_q, const CUtensorMap& tw,
                           const CUtensorMap& ts, const CUtensorMap& ta, const lq::GemmArgs& a, cudaStream_t st) {
-  if (dq == 0) return launch_gemm<I32>(s, tx, x_q, tw, ts, ta, a, st);
+  if (dq == 0) return launch_gemm<I32 ? kOutI32 : kOutBf16>(s, tx, x_q, tw, ts, ta, a, st);
   if (s.kind != kSchedTiles || s.cs != 4) return LQ_ERR_UNSUPPORTED_SHAPE;
   switch (s.bt * 4 + dq) {
     case 16 * 4 + 1: return launch_abl_t<16, 4, I32, 1>(s, tx, x_q, tw, ts, ta, a, st);
@@ -449,7 +458,7 @@ lq_status launch_ablation(const Schedule& s, int dq, const CUtensorMap& tx, cons
 lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
                     const uint8_t* a_u8, const float* s_c, void* out, int M, int N, int K, int group,
                     void* workspace, size_t ws_bytes, int block_t, int schedule, int split_k, int grid,
-                    bool out_i32, void* stream, int dq = 0) {
+                    bool out_i32, void* stream, int dq = 0, bool swiglu = false) {
   lq_status st = check_gemm_shape(M, N, K, group);
   if (st != LQ_OK) return st;
   if (!valid_schedule(M, block_t, schedule, split_k, grid)) return LQ_ERR_INVALID_ARG;
@@ -461,7 +470,14 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
-  const Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms);
+  Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms);
+  if (swiglu) {
+    // the SwiGLU epilogue runs on the tile kernel's cluster schedules and the
+    // CTA-pair kernel: a persistent choice becomes one cluster per tile
+    if (s.kind == kSchedStreamK || (s.kind == kSchedPersistent && schedule == kSchedPersistent))
+      return LQ_ERR_UNSUPPORTED_SHAPE;
+    if (s.kind == kSchedPersistent) s = make_schedule(M, N, K, lq::kPBT, kSchedTiles, 0, 0, dev->sms);
+  }
   st = check_schedule_shape(s, K);
   if (st != LQ_OK) return st;
   if (s.split) {
@@ -502,8 +518,9 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   if (dq != 0)
     return out_i32 ? launch_ablation<true>(s, dq, tx, x_q, tw, ts, ta, a, cs)
                    : launch_ablation<false>(s, dq, tx, x_q, tw, ts, ta, a, cs);
-  return out_i32 ? launch_gemm<true>(s, tx, x_q, tw, ts, ta, a, cs)
-                 : launch_gemm<false>(s, tx, x_q, tw, ts, ta, a, cs);
+  if (swiglu) return launch_gemm<kOutSwiglu>(s, tx, x_q, tw, ts, ta, a, cs);
+  return out_i32 ? launch_gemm<kOutI32>(s, tx, x_q, tw, ts, ta, a, cs)
+                 : launch_gemm<kOutBf16>(s, tx, x_q, tw, ts, ta, a, cs);
 }
 
 // ---------------------------------------- fused activation quantization
@@ -699,6 +716,21 @@ lq_status lq_w4a8_gemm(const int8_t* x_q, const float* s_x, const uint8_t* qw, c
                        void* workspace, size_t workspace_bytes, void* stream) {
   return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes, 0, 0,
                    0, 0, false, stream);
+}
+
+lq_status lq_w4a8_gemm_swiglu(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                              const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K, int group,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes, 0, 0, 0, 0,
+                   false, stream, 0, true);
+}
+
+lq_status lq_w4a8_gemm_swiglu_ex(const int8_t* x_q, const float* s_x, const uint8_t* qw, const uint8_t* s_u8,
+                                 const uint8_t* a_u8, const float* s_c, void* out_bf16, int M, int N, int K, int group,
+                                 void* workspace, size_t workspace_bytes, int block_t, int schedule, int split_k,
+                                 int grid, void* stream) {
+  return gemm_impl(x_q, s_x, qw, s_u8, a_u8, s_c, out_bf16, M, N, K, group, workspace, workspace_bytes, block_t,
+                   schedule, split_k, grid, false, stream, 0, true);
 }
 
 lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* s_u8, const uint8_t* a_u8,
@@ -918,8 +950,8 @@ lq_status grouped_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, c
   a.m_off = m_off;
   a.groups = groups;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  return out_i32 ? launch_gemm<true>(s, tx, x_q, tw, ts, ta, a, cs)
-                 : launch_gemm<false>(s, tx, x_q, tw, ts, ta, a, cs);
+  return out_i32 ? launch_gemm<kOutI32>(s, tx, x_q, tw, ts, ta, a, cs)
+                 : launch_gemm<kOutBf16>(s, tx, x_q, tw, ts, ta, a, cs);
 }
 
 }  // namespace

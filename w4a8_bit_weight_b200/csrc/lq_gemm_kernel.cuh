@@ -283,6 +283,40 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& p, int m_first, int 
   }
 }
 
+// SwiGLU epilogue of an interleaved gate/up pair: weight row 2j is gate
+// channel j, row 2j + 1 up channel j, so the gate and up values of an output
+// column sit in lanes 2i and 2i + 1 of a warp.  silu(g) = g / (1 + exp(-g))
+// in IEEE fp32 steps (expf: CUDA's, within 2 ulp), one bf16 rounding.
+__device__ __forceinline__ float silu_f32(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, expf(-g))); }
+
+// For a token pair (t, t + 1) whose fp32 values in this lane are y0, y1 (gate
+// values in even lanes, up values in odd lanes): the even lane returns the
+// output of token t, the odd lane that of token t + 1.  Every lane must call it.
+__device__ __forceinline__ float swiglu_pair(float y0, float y1) {
+  const bool odd = threadIdx.x & 1;
+  const float other = __shfl_xor_sync(0xffffffffu, odd ? y0 : y1, 1);  // partner's value of this lane's token
+  return odd ? __fmul_rn(silu_f32(other), y1) : __fmul_rn(silu_f32(y0), other);
+}
+
+// Writes TC tokens [m_first, m_first + TC) of output column n / 2 from the
+// accumulators v of weight row n (SwiGLU; see swiglu_pair).  Every lane must call it.
+template <int TC>
+__device__ __forceinline__ void store_chunk_swiglu(const GemmArgs& p, int m_first, int mend, int n, bool n_ok,
+                                                   const uint32_t* v, float sx_lane, float sc) {
+  const bool odd = threadIdx.x & 1;
+  const int ld = p.N >> 1;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m_first * ld + (n >> 1);
+#pragma unroll
+  for (int i = 0; i < TC; i += 2) {
+    const float y0 = __fmul_rn(__int2float_rn((int32_t)v[i]), __fmul_rn(__shfl_sync(0xffffffffu, sx_lane, i), sc));
+    const float y1 =
+        __fmul_rn(__int2float_rn((int32_t)v[i + 1]), __fmul_rn(__shfl_sync(0xffffffffu, sx_lane, i + 1), sc));
+    const float out = swiglu_pair(y0, y1);
+    const int t = i + (odd ? 1 : 0);
+    if (n_ok && m_first + t < mend) o[(size_t)t * ld] = __float2bfloat16_rn(out);
+  }
+}
+
 // Output element from an accumulator and the token's scale s_x[m] (given).
 template <bool OUT_I32>
 __device__ __forceinline__ void store_out_sx(const GemmArgs& p, int m, int n, int32_t acc, float sx, float sc) {
@@ -340,7 +374,7 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[W]) {
 // the expansion warps quantize them (per-token symmetric INT8, the same
 // arithmetic as quantize_act_kernel) straight into the swizzled activation
 // tiles; the row maxima are combined over the cluster through DSMEM.
-template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0, int EG = 1>
+template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0, int EG = 1, bool SWI = false>
 __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCols == 256 ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_x3,
                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
@@ -348,6 +382,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
   using C = GemmCfg<BT, CS, DQ>;
   constexpr int kEG = EG;  // expansion groups of this variant
   static_assert(EG == 1 || (EG == 2 && !FQ && CS >= 1), "two expansion groups: cluster schedules, no fused quantization");
+  static_assert(!SWI || (!OUT_I32 && !FQ && DQ == 0 && CS >= 1), "SwiGLU epilogue: bf16 output of cluster schedules");
   static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
   static_assert(DQ == 0 || (!FQ && CS >= 1), "ablation variants: plain tile schedules only");
   constexpr int S = C::kStages;
@@ -1171,18 +1206,22 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
                 }
               }
               const float sx_chunk = (kSxRegs > 1 && c0 >= 32) ? sxr[kSxRegs - 1] : sxr[0];  // tokens c0 .. c0 + 31
+              if constexpr (SWI) {
+                store_chunk_swiglu<TCH>(p, sx0 + c0, mend, n, n_ok, acc, sx_chunk, sc);
+              } else {
 #pragma unroll
-              for (int i = 0; i < TCH; ++i) {
-                const int ti = c0 + i;  // token of the slice
-                const int m = sx0 + ti;
-                float sxm = 0.0f;
-                if constexpr (!OUT_I32) sxm = __shfl_sync(0xffffffffu, sx_chunk, i);
-                if (m < mend && n_ok) {
-                  if constexpr (OUT_I32) {
-                    reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)acc[i];
-                  } else {
-                    const float y = __fmul_rn(__int2float_rn((int32_t)acc[i]), __fmul_rn(sxm, sc));
-                    reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
+                for (int i = 0; i < TCH; ++i) {
+                  const int ti = c0 + i;  // token of the slice
+                  const int m = sx0 + ti;
+                  float sxm = 0.0f;
+                  if constexpr (!OUT_I32) sxm = __shfl_sync(0xffffffffu, sx_chunk, i);
+                  if (m < mend && n_ok) {
+                    if constexpr (OUT_I32) {
+                      reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)acc[i];
+                    } else {
+                      const float y = __fmul_rn(__int2float_rn((int32_t)acc[i]), __fmul_rn(sxm, sc));
+                      reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
+                    }
                   }
                 }
               }
@@ -1209,7 +1248,10 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
               tmem_load_cols<CH>(t_lane + cc * CH, v);
             }
             if (whole) {
-              store_chunk<OUT_I32, CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
+              if constexpr (SWI)
+                store_chunk_swiglu<CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
+              else
+                store_chunk<OUT_I32, CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
             } else {
 #pragma unroll
               for (int i = 0; i < CH; ++i) {

@@ -157,7 +157,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-template <bool OUT_I32>
+template <bool OUT_I32, bool SWI = false>
 __global__ void __launch_bounds__(kQThreads, 1)
     w4a8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                           const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_a,
@@ -471,6 +471,45 @@ __global__ void __launch_bounds__(kQThreads, 1)
             const int m = mb + cc * 32 + i;
             if (m < mend && n_ok) reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)v[i];
           }
+        }
+      } else if constexpr (SWI) {
+        // SwiGLU of the interleaved gate/up rows (swiglu_pair): this lane's
+        // output of each token pair (the even token in even lanes, the odd one
+        // in odd lanes) as bf16 in registers first, the accumulator handed back
+        // before any global store.
+        uint32_t pk[32];  // pk[q / 2]: outputs of token pairs q (low half) and q + 1 (high half)
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(t_lane + e * 128 + cc * 16, v);
+          const float sxl = sx4[cc >> 1];
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            const int src = (cc & 1) * 16 + i;
+            const float y0 = __fmul_rn(__int2float_rn((int32_t)v[i]), __fmul_rn(__shfl_sync(0xffffffffu, sxl, src), sc));
+            const float y1 =
+                __fmul_rn(__int2float_rn((int32_t)v[i + 1]), __fmul_rn(__shfl_sync(0xffffffffu, sxl, src + 1), sc));
+            const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(swiglu_pair(y0, y1)));
+            const int q = 8 * cc + i / 2;  // token pair of the warp's 128
+            if (q & 1)
+              pk[q >> 1] |= b << 16;
+            else
+              pk[q >> 1] = b;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_on_leader(accempty, crank);
+        const bool odd = lane & 1;
+        const int ld = p.N >> 1;
+        const bool pair_ok = n_ok;  // N is a multiple of 16: a gate row and its up row are both valid or not
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (n >> 1);
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          const int m = mb + 2 * q + (odd ? 1 : 0);
+          const uint32_t h = (q & 1) ? (pk[q >> 1] >> 16) : (pk[q >> 1] & 0xFFFFu);
+          if (m < mend && pair_ok) o[(size_t)m * ld] = __ushort_as_bfloat16((unsigned short)h);
         }
       } else {
         // All four chunks to packed bf16 in registers first, so the accumulator
