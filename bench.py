@@ -1,6 +1,6 @@
 """Benchmark of the B200 LiquidQuant W4A8 GEMM path.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|mlp_up|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill|mlp_up|down_sweep|tiny]
     python bench.py --impl reference ...      # the CPU oracle on the host cores
 
 One step is one pass of the per-forward hot path over one batch: for every
@@ -18,6 +18,13 @@ launch streams its weights from HBM.  The GEMM's own duration per launch (the
 roofline's denominator) comes from a second graph of K back-to-back GEMM calls
 per M, timed the same way: the launches overlap through programmatic dependent
 launch exactly as in the step, and replay time / K is the time per launch.
+
+The default (decode) run also measures, in the same process: the prefill
+layer, a dense INT8 ceiling (torch._int_mm at 8192^3), the MLP up/gate layer
+and the down-projection sweep (every M of both), the fused SwiGLU gate/up pair
+against two GEMMs plus a separate activation, the grouped GEMM, the
+dequantization ablation and the W4 x FP8 variant -- each as side objects of
+the JSON line.
 
 With --gpus N > 1 (launched by torchrun) every rank runs an independent
 replica (the path has no exchange step); the time is the max over ranks and
@@ -54,7 +61,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "mlp_up", "tiny"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "mlp_up", "down_sweep", "tiny"])
     ap.add_argument("--soak-s", type=float, default=1.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -427,6 +434,8 @@ def run_ours(args, rank, world, local_rank):
                         else "two_launches"} for M in Ms}}
     res["int8_peak_tops"] = int8_peak
     if args.workload == "decode" and not args.no_secondary:
+        ceil = int8_ceiling(dev)
+        res["int8_ceiling"] = ceil
         pre = secondary_workload("prefill", dev)
         g = pre["4096"]
         pre["roofline"] = {"bound": "tensor", "kernel": "w4a8_gemm_pair_kernel", "achieved": g["gemm_tops"],
@@ -434,7 +443,13 @@ def run_ours(args, rank, world, local_rank):
                            "peak_source": f"{pk_src}: {INT8_OVER_BF16:g} x bf16 burst",
                            "frac_of_nominal_4500": g["gemm_tops"] / 4500.0,
                            "traffic": ncu_traffic("prefill")}
+        if "tops" in ceil:
+            pre["roofline"]["measured_int8_ceiling_tops"] = ceil["tops"]
+            pre["roofline"]["frac_of_measured_int8_ceiling"] = g["gemm_tops"] / ceil["tops"]
         res["prefill"] = pre
+        res["mlp_up"] = shape_sweep("mlp_up", dev, hbm_peak, int8_peak)
+        res["down_sweep"] = shape_sweep("down_sweep", dev, hbm_peak, int8_peak)
+        res["swiglu"] = swiglu_side(dev, hbm_peak, int8_peak)
         res["grouped"] = grouped_side(dev, int8_peak, hbm_peak)
         res["ablation"] = ablation_side(dev, hbm_peak)
         try:
@@ -608,6 +623,137 @@ def w4f8_side(dev, hbm_peak, n=40):
         res[str(M)] = {"us": us, "gbs": byts / (us * 1e-6) / 1e9, "frac_of_hbm": byts / (us * 1e-6) / 1e9 / hbm_peak}
         del g
     return res
+
+
+def _graph_us(stream, dev, fn, n, reps=3):
+    """Median over `reps` replays of a CUDA graph of n calls of fn(i), us per call
+    (the graph is replayed once untimed first: its first launch also uploads it)."""
+    for i in range(2):
+        fn(i)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(1e3 * e0.elapsed_time(e1) / n)
+    del g
+    return sorted(ts)[len(ts) // 2]
+
+
+def _roofline(M, N, K, us, hbm_peak, int8_peak):
+    byts = gemm_bytes(M, N, K)
+    ops = 2.0 * M * N * K
+    t_hbm, t_tc = byts / (hbm_peak * 1e9), ops / (int8_peak * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    return {"us": us, "gbs": byts / (us * 1e-6) / 1e9, "tops": ops / (us * 1e-6) / 1e12, "bound": bound,
+            "frac": max(t_hbm, t_tc) / (us * 1e-6)}
+
+
+def shape_sweep(workload, dev, hbm_peak, int8_peak, n=20):
+    """Back-to-back lq_w4a8_gemm launches of each M of a workload (its N, K, seeded
+    weights and activations), weights rotating over L2-cold copies; us per launch,
+    GB/s of algorithmic bytes, TOPS, and the fraction of the larger of the HBM time
+    and the INT8 tensor time."""
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+    w = synth.WORKLOADS[workload]
+    X, W = synth.make_workload(w)
+    qw, s_u8, a_u8, s_c = lq.lq_quantize_weights(W.to(dev))
+    wset = qw.numel() + 2 * s_u8.numel() + 4 * s_c.numel()
+    n_sets = min(48, max(4, int(np.ceil(3 * L2_BYTES / wset))))
+    sets = [(qw, s_u8, a_u8, s_c)] + [(qw.clone(), s_u8.clone(), a_u8.clone(), s_c.clone())
+                                      for _ in range(n_sets - 1)]
+    stream = torch.cuda.Stream(dev)
+    res = {"workload": w.note, "how": f"{n} back-to-back lq_w4a8_gemm calls per M in one CUDA graph, "
+                                      f"weights rotating over {n_sets} copies; roofline = max(HBM time at "
+                                      f"{hbm_peak:.0f} GB/s, INT8 time at {int8_peak:.0f} TOPS)"}
+    Xd = X.to(dev)
+    for M in w.Ms:
+        xq, sx = lq.lq_quantize_act(Xd[:M])
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
+        with torch.cuda.stream(stream):
+            us = _graph_us(stream, dev, lambda i: lq.lq_w4a8_gemm(xq, sx, *sets[i % n_sets], out=out), n)
+        res[str(M)] = _roofline(M, w.N, w.K, us, hbm_peak, int8_peak)
+        del xq, sx, out
+    if lq.lq_get_device_error(dev) != 0:
+        raise RuntimeError(f"device error in the {workload} sweep")
+    return res
+
+
+def swiglu_side(dev, hbm_peak, int8_peak, n=20):
+    """The MLP up/gate layer as a gated FFN pair: F = 14336 gate + 14336 up channels,
+    K = 4096, M = 16 / 256 / 4096.  One lq_w4a8_gemm_swiglu launch on the interleaved
+    [2F, K] weights against two lq_w4a8_gemm launches (gate, up) plus the separate
+    activation silu(gate) * up (torch, bf16) -- the same work, unfused."""
+    import w4a8_bit_weight_b200 as lq
+    from w4a8_bit_weight_b200 import synth
+    w = synth.WORKLOADS["mlp_up"]
+    F, K = w.N, w.K
+    X, W = synth.make_problem(max(w.Ms), 2 * F, K, seed=31, n_outliers=41)
+    qw, s_u8, a_u8, s_c = lq.lq_quantize_weights(W.to(dev))
+    # gate rows are the even rows, up rows the odd ones: the same weights, unfused
+    qg, sg, ag, cg = lq.lq_quantize_weights(W[0::2].contiguous().to(dev))
+    qu, su, au, cu = lq.lq_quantize_weights(W[1::2].contiguous().to(dev))
+    wset = 2 * (qw.numel() + 2 * s_u8.numel() + 4 * s_c.numel())
+    n_sets = min(16, max(2, int(np.ceil(3 * L2_BYTES / wset))))
+    fused = [(qw, s_u8, a_u8, s_c)] + [(qw.clone(), s_u8.clone(), a_u8.clone(), s_c.clone()) for _ in range(n_sets - 1)]
+    split = [((qg, sg, ag, cg), (qu, su, au, cu))] + [
+        ((qg.clone(), sg.clone(), ag.clone(), cg.clone()), (qu.clone(), su.clone(), au.clone(), cu.clone()))
+        for _ in range(n_sets - 1)]
+    stream = torch.cuda.Stream(dev)
+    res = {"workload": f"gated FFN up/gate pair F={F} (+{F}) K={K}, interleaved weights",
+           "how": f"{n} back-to-back calls per M in one CUDA graph, weights rotating over {n_sets} copies; "
+                  "unfused = gate GEMM + up GEMM + torch silu(g)*u on their bf16 outputs"}
+    Xd = X.to(dev)
+    for M in w.Ms:
+        xq, sx = lq.lq_quantize_act(Xd[:M])
+        out = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+        g_out = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+        u_out = torch.empty(M, F, dtype=torch.bfloat16, device=dev)
+
+        def unfused(i):
+            gw, uw = split[i % n_sets]
+            lq.lq_w4a8_gemm(xq, sx, *gw, out=g_out)
+            lq.lq_w4a8_gemm(xq, sx, *uw, out=u_out)
+            torch.mul(torch.nn.functional.silu(g_out), u_out, out=out)
+
+        with torch.cuda.stream(stream):
+            us_f = _graph_us(stream, dev, lambda i: lq.lq_w4a8_gemm_swiglu(xq, sx, *fused[i % n_sets], out=out), n)
+            us_u = _graph_us(stream, dev, unfused, n)
+        r = _roofline(M, 2 * F, K, us_f, hbm_peak, int8_peak)
+        # the fused output is F columns, not 2F: count its bytes as written
+        byts = gemm_bytes(M, 2 * F, K) - 2 * M * F
+        r["gbs"] = byts / (us_f * 1e-6) / 1e9
+        res[str(M)] = {"fused_us": us_f, "unfused_us": us_u, "speedup": us_u / us_f, "fused": r}
+        del xq, sx, out, g_out, u_out
+    if lq.lq_get_device_error(dev) != 0:
+        raise RuntimeError("device error in the SwiGLU measurement")
+    return res
+
+
+def int8_ceiling(dev, size=8192, n=10):
+    """A dense INT8 GEMM ceiling measured in the same run: torch._int_mm (cuBLASLt)
+    at size^3, as back-to-back calls in one CUDA graph.  None if it does not run."""
+    try:
+        a = torch.randint(-127, 128, (size, size), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (size, size), dtype=torch.int8, device=dev)
+        c = torch.empty(size, size, dtype=torch.int32, device=dev)
+        stream = torch.cuda.Stream(dev)
+        with torch.cuda.stream(stream):
+            us = _graph_us(stream, dev, lambda i: torch._int_mm(a, b, out=c), n)
+        return {"tops": 2.0 * size ** 3 / (us * 1e-6) / 1e12, "us": us,
+                "how": f"torch._int_mm {size}^3, {n} back-to-back calls in one CUDA graph"}
+    except Exception as ex:  # a side measurement never takes the bench line down
+        return {"error": str(ex)[:200]}
 
 
 def secondary_workload(name, dev, steps=20):
