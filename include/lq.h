@@ -394,9 +394,13 @@ LQ_API lq_status lq_w4a8_grouped_gemm_ex(const int8_t* x_q, const float* s_x, co
  *   (the tensor's maximum is gathered in s_x's word first).  K % 16 == 0.
  * lq_w4f8_gemm -- out[m,n] = bf16(acc * (s_x[0] * s_w[n])), acc the fp32
  *   sum over k of e4m3(x)[m,k] * q[n,k] computed by tcgen05.mma
- *   kind::f8f6f4 (the products are exact, the fp32 accumulation order is the
- *   tensor core's).  One CTA per 128-row x 16- or 128-token tile.  Shape and
- *   alignment rules as lq_w4a8_gemm (no group, no workspace).
+ *   kind::f8f6f4 (the products are exact; the fp32 accumulation order is the
+ *   tensor core's within a CTA's K-slice, and split-K partial sums are added
+ *   in a fixed order, so repeated calls give identical bits).  The schedule
+ *   is lq_w4a8_gemm's cluster form for 16-, 64- or 128-token tiles (M <= 16,
+ *   <= 64, above): a cluster of CTAs per 128-row tile, split over K and
+ *   reduce-scattered through distributed shared memory.  Shape and alignment
+ *   rules as lq_w4a8_gemm (no group, no workspace).  Allocates nothing.
  */
 LQ_API lq_status lq_quantize_weights_w4(const void* W_bf16, int N, int K, uint8_t* qw4, float* s_w, void* stream);
 LQ_API lq_status lq_quantize_act_f8(const void* X_bf16, int M, int K, uint8_t* x_f8, float* s_x, void* stream);

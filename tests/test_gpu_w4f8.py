@@ -25,8 +25,12 @@ def _u16(t):
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+# the schedule forms: 16-token tiles with 1, 2, 4 and 8 CTAs per cluster (two
+# expansion groups, two MMA issuers, the overflow block at M = 1..16,
+# N = K = 4096), 64- and 128-token tiles, ragged N, K and M tails
 @pytest.mark.parametrize("M,N,K", [(16, 256, 512), (5, 384, 1024), (130, 256, 768), (16, 4096, 4096),
-                                   (200, 4096, 1024)])
+                                   (1, 4096, 4096), (200, 4096, 1024), (16, 1024, 4096), (40, 1024, 2048),
+                                   (3, 400, 640), (300, 512, 1024), (64, 2048, 128)])
 def test_w4f8_matches_oracle(M, N, K):
     torch.cuda.set_device(0)
     X, W = synth.make_problem(M, N, K, seed=M + N + K + 5, n_outliers=3)
@@ -63,3 +67,41 @@ def test_w4f8_zero_activations():
     out = lq.lq_w4f8_gemm(x_f8, s_x, qw4, s_w)
     torch.cuda.synchronize()
     assert float(s_x.cpu()[0]) == 1.0 and not x_f8.any() and not (out != 0).any()
+
+
+def test_w4f8_repeatable():
+    """Split-K partial sums are added in a fixed order: two calls give the same bits."""
+    torch.cuda.set_device(0)
+    X, W = synth.make_problem(16, 4096, 4096, seed=11, n_outliers=3)
+    qw4, s_w = lq.lq_quantize_weights_w4(W.to(DEV))
+    x_f8, s_x = lq.lq_quantize_act_f8(X.to(DEV))
+    a = lq.lq_w4f8_gemm(x_f8, s_x, qw4, s_w)
+    b = lq.lq_w4f8_gemm(x_f8, s_x, qw4, s_w)
+    torch.cuda.synchronize()
+    assert lq.lq_get_device_error() == 0
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_w4f8_all_codes():
+    """Every INT4 code, -8 included, against exact sums: weights whose codes cycle
+    through 0..15 (u = q + 8) and activations of +-1 in e4m3, so that acc is an
+    exactly representable integer and the output is bf16(acc * s_x * s_w[n])."""
+    torch.cuda.set_device(0)
+    M, N, K = 16, 256, 1024
+    rng = np.random.default_rng(7)
+    u = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    # the LiquidQuant nibble layout: byte b of word j = u[8j + b] | u[8j + 4 + b] << 4
+    g = u.reshape(N, K // 8, 2, 4)
+    qw4 = (g[:, :, 0, :] | (g[:, :, 1, :] << 4)).reshape(N, K // 2).astype(np.uint8)
+    xs = rng.choice(np.array([0x38, 0xB8, 0x00], dtype=np.uint8), size=(M, K))  # +1, -1, 0 in e4m3
+    s_w = rng.uniform(0.5, 2.0, size=N).astype(np.float32)
+    s_x = np.array([0.25], dtype=np.float32)
+    out = lq.lq_w4f8_gemm(torch.from_numpy(xs).to(DEV), torch.from_numpy(s_x).to(DEV),
+                          torch.from_numpy(qw4).to(DEV), torch.from_numpy(s_w).to(DEV))
+    torch.cuda.synchronize()
+    assert lq.lq_get_device_error() == 0
+    xv = np.where(xs == 0x38, 1.0, np.where(xs == 0xB8, -1.0, 0.0))
+    acc = xv @ (u.astype(np.float64) - 8).T
+    ref = torch.from_numpy((acc * (np.float32(s_x[0]) * s_w).astype(np.float64)[None, :]).astype(np.float32))
+    want = ref.to(torch.bfloat16).view(torch.int16).numpy()
+    np.testing.assert_array_equal(_u16(out).view(np.int16), want)

@@ -975,6 +975,79 @@ lq_status lq_w4a8_grouped_gemm(const int8_t* x_q, const float* s_x, const uint8_
 }  // extern "C"
 
 // ------------------------------------------------------------ W4 x FP8
+namespace {
+
+// The tile kernel's KIND 1 on its cluster schedules: 16-, 64- or 128-token
+// tiles, the split and the expansion groups chosen as for W4A8.  The weight
+// map stands in for the scale / offset maps, which KIND 1 never reads.
+template <int BT, int CS, int EG>
+lq_status launch_f8_tg(const Schedule& s, const CUtensorMap& tx, const void* x_f8, const CUtensorMap& tw,
+                       const lq::GemmArgs& a, cudaStream_t st) {
+  using C = lq::GemmCfg<BT, CS>;
+  auto kern = lq::w4a8_gemm_kernel<BT, CS, false, false, 0, EG, false, 1>;
+  CUtensorMap tx3;
+  if (!make_tile_x3<BT, CS, 0>(&tx3, tx, x_f8, a)) return LQ_ERR_CUDA;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+    return LQ_ERR_CUDA;
+  return launch_ex(kern, s.grid, lq::gemm_threads(EG), C::kSmemBytes, CS, pdl_enabled(), st, tx, tx3, tw, tw, tw, a);
+}
+
+template <int BT, int CS>
+lq_status launch_f8_t(const Schedule& s, const CUtensorMap& tx, const void* x_f8, const CUtensorMap& tw,
+                      const lq::GemmArgs& a, cudaStream_t st) {
+  if constexpr (BT == 16) {
+    if ((s.KB + CS - 1) / CS <= lq::GemmCfg<BT, CS>::kStages) return launch_f8_tg<BT, CS, 2>(s, tx, x_f8, tw, a, st);
+  }
+  return launch_f8_tg<BT, CS, 1>(s, tx, x_f8, tw, a, st);
+}
+
+template <int BT>
+lq_status launch_f8_bt(const Schedule& s, const CUtensorMap& tx, const void* x_f8, const CUtensorMap& tw,
+                       const lq::GemmArgs& a, cudaStream_t st) {
+  switch (s.cs) {
+    case 1: return launch_f8_t<BT, 1>(s, tx, x_f8, tw, a, st);
+    case 2: return launch_f8_t<BT, 2>(s, tx, x_f8, tw, a, st);
+    case 4: return launch_f8_t<BT, 4>(s, tx, x_f8, tw, a, st);
+    case 8:
+      if constexpr (BT <= 32) return launch_f8_t<BT, 8>(s, tx, x_f8, tw, a, st);
+      break;
+  }
+  return LQ_ERR_INVALID_ARG;
+}
+
+lq_status w4f8_impl(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4, const float* s_w, void* out, int M,
+                    int N, int K, int sms, cudaStream_t st) {
+  const int bt = M <= 16 ? 16 : M <= 64 ? 64 : 128;
+  const Schedule s = make_schedule(M, N, K, bt, kSchedTiles, 0, 0, sms);
+  if (s.tiles * s.cs > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap tx, tw;
+  if (!make_map_u8(&tx, x_f8, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, (uint32_t)bt,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&tw, qw4, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, lq::kBlockK / 2, lq::kBlockN,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return LQ_ERR_CUDA;
+  lq::GemmArgs a;
+  a.x_bf16 = nullptr;
+  a.s_x = s_x;
+  a.s_c = s_w;
+  a.out = out;
+  a.ws = nullptr;
+  a.ticket = nullptr;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = s.tiles_m;
+  a.KB = s.KB;
+  a.U = s.U;
+  switch (bt) {
+    case 16: return launch_f8_bt<16>(s, tx, x_f8, tw, a, st);
+    case 64: return launch_f8_bt<64>(s, tx, x_f8, tw, a, st);
+    default: return launch_f8_bt<128>(s, tx, x_f8, tw, a, st);
+  }
+}
+
+}  // namespace
+
 extern "C" {
 
 lq_status lq_quantize_weights_w4(const void* W_bf16, int N, int K, uint8_t* qw4, float* s_w, void* stream) {
@@ -1023,35 +1096,7 @@ lq_status lq_w4f8_gemm(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
-  const int bt = M <= 16 ? 16 : 128;
-  const int tiles_m = (M + bt - 1) / bt, tiles_n = (N + lq::kBlockN - 1) / lq::kBlockN;
-  if ((long long)tiles_m * tiles_n > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap tx, tw;
-  if (!make_map_u8(&tx, x_f8, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128u, (uint32_t)bt, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_u8(&tw, qw4, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 64u, 128u, CU_TENSOR_MAP_SWIZZLE_64B))
-    return LQ_ERR_CUDA;
-  lq::F8Args a;
-  a.s_x = s_x;
-  a.s_w = s_w;
-  a.out = static_cast<__nv_bfloat16*>(out_bf16);
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.tiles_m = tiles_m;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const int grid = tiles_m * tiles_n;
-  if (bt == 16) {
-    auto kern = lq::w4f8_gemm_kernel<16>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::F8Cfg<16>::kSmemBytes) !=
-        cudaSuccess)
-      return LQ_ERR_CUDA;
-    return launch_ex(kern, grid, lq::kF8Threads, lq::F8Cfg<16>::kSmemBytes, 1, pdl_enabled(), cs, tx, tw, a);
-  }
-  auto kern = lq::w4f8_gemm_kernel<128>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lq::F8Cfg<128>::kSmemBytes) !=
-      cudaSuccess)
-    return LQ_ERR_CUDA;
-  return launch_ex(kern, grid, lq::kF8Threads, lq::F8Cfg<128>::kSmemBytes, 1, pdl_enabled(), cs, tx, tw, a);
+  return w4f8_impl(x_f8, s_x, qw4, s_w, out_bf16, M, N, K, dev->sms, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -299,6 +299,35 @@ __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// kind::f8f6f4 (e4m3 A and B, fp32 D) with A in tensor memory / in shared memory.
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::f8f6f4 instruction descriptor: fp32 D, e4m3 A and B, both K-major,
+// M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_f8(int n) {
+  return (1u << 4)                        // D format: f32
+         | (0u << 7) | (0u << 10)         // A, B: e4m3
+         | (uint32_t(n >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+}
+
 // Instruction descriptor for kind::i8: signed A and B, int32 D, both K-major,
 // M = 128, N = n (multiple of 16, 16..256).
 __host__ __device__ constexpr uint32_t idesc_i8(int n) {
@@ -412,6 +441,35 @@ __device__ __forceinline__ void lqq_expand_word(uint32_t w, uint32_t s, uint32_t
                                                 uint32_t& hi) {
   lo = ((w & 0x0F0F0F0Fu) * s + a4) ^ 0x80808080u;
   hi = (((w >> 4) & 0x0F0F0F0Fu) * s + a4) ^ 0x80808080u;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Eight symmetric INT4 codes of one packed word (u = q + 8, code k in byte
+// k % 4, high nibble for k >= 4) as eight e4m3 bytes in code order: codes 0-3
+// in `lo`, 4-7 in `hi`.  Every integer in [-8, 7] is an e4m3 value, so this
+// is exact.  Byte permutes serve as 8-entry tables, indexed by a nibble's low
+// three bits; a selector nibble with bit 3 set fills the byte with the top
+// bit of the entry instead, and both tables keep that bit clear:
+//   table P (e4m3 of 0..7), selectors u ^ 8: u >= 8 reads e4m3(u - 8),
+//     u < 8 reads 0;
+//   table N (e4m3 of -8..-1 without the sign bit), selectors u: u < 8 reads
+//     |e4m3(u - 8)|, u >= 8 reads 0.
+// The selectors of one 16-bit half are codes (0, 4, 1, 5) or (2, 6, 3, 7), so
+// two more permutes put the bytes in code order; the sign (u < 8) is bit 3 of
+// the code, negated and moved to bit 7 of its byte.
+__device__ __forceinline__ void w4_word_to_e4m3(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  constexpr uint32_t kP0 = 0x44403800u, kP1 = 0x4E4C4A48u;  // e4m3(0..3), e4m3(4..7)
+  constexpr uint32_t kN0 = 0x4A4C4E50u, kN1 = 0x38404448u;  // |e4m3(-8..-5)|, |e4m3(-4..-1)|
+  const uint32_t wf = w ^ 0x88888888u;
+  const uint32_t r0 = prmt(kP0, kP1, wf) | prmt(kN0, kN1, w);               // codes 0, 4, 1, 5
+  const uint32_t r1 = prmt(kP0, kP1, wf >> 16) | prmt(kN0, kN1, w >> 16);   // codes 2, 6, 3, 7
+  lo = prmt(r0, r1, 0x6420u) | (~(w << 4) & 0x80808080u);
+  hi = prmt(r0, r1, 0x7531u) | (~w & 0x80808080u);
 }
 
 // The same eight values one at a time (nibble extract, IMAD, XOR, byte insert

@@ -50,8 +50,14 @@
 //
 // Also here: the grouped form (GemmArgs::m_off, one weight matrix per group
 // of token rows, each cluster finding its group on the device), the fused
-// activation quantization (FQ) and the variants of the dequantization
-// ablation (DQ).
+// activation quantization (FQ), the variants of the dequantization ablation
+// (DQ), and the W4 x FP8 variant (KIND 1, FireQ page, abstract): symmetric
+// INT4 weights expanded to e4m3 (w4_word_to_e4m3, exact), e4m3 activations
+// with one scale for the tensor, tcgen05.mma kind::f8f6f4 into fp32
+// accumulators.  The schedules, the pipeline and the reduce-scatter are the
+// same; the partial sums are fp32, added in a fixed order, so every run of
+// one schedule gives the same bits (different schedules may differ in the
+// last place of the fp32 sums).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -258,11 +264,41 @@ __device__ __forceinline__ uint32_t quant_quad_i8(uint32_t w01, uint32_t w23, fl
   return r;
 }
 
+// Accumulator words: int32 sums (W4A8) or fp32 sums (W4 x FP8).
+template <bool F8>
+__device__ __forceinline__ float acc_f32(uint32_t v) {
+  if constexpr (F8)
+    return __uint_as_float(v);
+  else
+    return __int2float_rn((int32_t)v);
+}
+template <bool F8>
+__device__ __forceinline__ uint32_t acc_add(uint32_t a, uint32_t b) {
+  if constexpr (F8)
+    return __float_as_uint(__fadd_rn(__uint_as_float(a), __uint_as_float(b)));
+  else
+    return a + b;
+}
+template <bool F8>
+__device__ __forceinline__ void mma_ts_k(uint32_t d, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  if constexpr (F8)
+    mma_f8_ts(d, a_tmem, b_desc, idesc, acc);
+  else
+    mma_i8_ts(d, a_tmem, b_desc, idesc, acc);
+}
+template <bool F8>
+__device__ __forceinline__ void mma_ss_k(uint32_t d, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  if constexpr (F8)
+    mma_f8_ss(d, a_desc, b_desc, idesc, acc);
+  else
+    mma_i8_ss(d, a_desc, b_desc, idesc, acc);
+}
+
 // Writes TC consecutive tokens [m_first, m_first + TC) of this thread's output
 // column n from the accumulators v.  sx_lane holds s_x[m_first + lane] (lanes
 // < TC).  The token scales are gathered first, so that the stores do not wait
 // on one another.  Every lane of the warp must call it.
-template <bool OUT_I32, int TC>
+template <bool OUT_I32, int TC, bool F8 = false>
 __device__ __forceinline__ void store_chunk(const GemmArgs& p, int m_first, int mend, int n, bool n_ok, const uint32_t* v,
                                             float sx_lane, float sc) {
   float scale[TC];
@@ -279,7 +315,7 @@ __device__ __forceinline__ void store_chunk(const GemmArgs& p, int m_first, int 
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)m_first * p.N + n;
 #pragma unroll
     for (int i = 0; i < TC; ++i)
-      if (i < mlim) o[(size_t)i * p.N] = __float2bfloat16_rn(__fmul_rn(__int2float_rn((int32_t)v[i]), scale[i]));
+      if (i < mlim) o[(size_t)i * p.N] = __float2bfloat16_rn(__fmul_rn(acc_f32<F8>(v[i]), scale[i]));
   }
 }
 
@@ -374,7 +410,11 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[W]) {
 // the expansion warps quantize them (per-token symmetric INT8, the same
 // arithmetic as quantize_act_kernel) straight into the swizzled activation
 // tiles; the row maxima are combined over the cluster through DSMEM.
-template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0, int EG = 1, bool SWI = false>
+//
+// KIND 1 (W4 x FP8): the tensor maps carry e4m3 activations and the packed
+// INT4 codes (no scale / offset tiles: tm_s and tm_a are never read); s_x is
+// the tensor's one scale, s_c the channel scales s_w.
+template <int BT, int CS, bool OUT_I32, bool FQ = false, int DQ = 0, int EG = 1, bool SWI = false, int KIND = 0>
 __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCols == 256 ? 2 : 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_x3,
                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
@@ -385,6 +425,11 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
   static_assert(!SWI || (!OUT_I32 && !FQ && DQ == 0 && CS >= 1), "SwiGLU epilogue: bf16 output of cluster schedules");
   static_assert(!FQ || (BT == 16 && CS >= 2), "fused activation quantization: 16-token tiles, split-K clusters");
   static_assert(DQ == 0 || (!FQ && CS >= 1), "ablation variants: plain tile schedules only");
+  static_assert(KIND == 0 || (KIND == 1 && !OUT_I32 && !FQ && DQ == 0 && !SWI && CS >= 1),
+                "W4 x FP8: bf16 output of cluster schedules");
+  constexpr bool F8 = (KIND == 1);
+  // bytes a weight stage's loads complete (W4 x FP8 has no scale / offset tiles)
+  constexpr uint32_t kTxW = F8 ? (uint32_t)C::kWBytes : C::kTxW;
   constexpr int S = C::kStages;
   constexpr int A = C::kSlots;
   // with as many TMEM slots as stages, block `it` uses stage and slot it % S:
@@ -507,8 +552,10 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
     fence_mbar_init();
     if (!FQ) tma_prefetch_desc(CS >= 1 ? &tm_x3 : &tm_x);
     tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_s);
-    tma_prefetch_desc(&tm_a);
+    if (!F8) {
+      tma_prefetch_desc(&tm_s);
+      tma_prefetch_desc(&tm_a);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -540,7 +587,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
   auto dual_issue = [&](int i) -> bool {
     bool ok = true;
     if (leader) {
-      constexpr uint32_t idesc = idesc_i8(BT);
+      constexpr uint32_t idesc = F8 ? idesc_f8(BT) : idesc_i8(BT);
       ok = mbar_wait(xfirst, 0, abort_flag);
       const int bl = ((total_u - 1 - i) & 1) ? total_u - 2 : total_u - 1;  // last block of this issuer
       if (ok && !(ovf && bl == A ? mbar_try_wait(smem_u32(ovfull), 0) : mbar_try_wait(smem_u32(&afull[bl]), 0)))
@@ -556,12 +603,12 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
             const uint64_t adesc = smem_desc_k_sw128(smem_u32(wring));
 #pragma unroll
             for (int j = 0; j < kBlockK / 32; ++j)
-              mma_i8_ss(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+              mma_ss_k<F8>(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
           } else {
             const uint32_t a_col = tmem_base + C::kAccCols + b * 32;
 #pragma unroll
             for (int j = 0; j < kBlockK / 32; ++j)
-              mma_i8_ts(d, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+              mma_ts_k<F8>(d, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
           }
         }
         tc_commit(accfull);
@@ -596,11 +643,13 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
     for (int i = 0; i < P; ++i, cw.next(KB, p.tiles_m)) {
       if (leader) {
         uint8_t* wb = wring + i * C::kWStage;
-        mbar_arrive_expect_tx(&wfull[i], C::kTxW);
+        mbar_arrive_expect_tx(&wfull[i], kTxW);
         const int wr = wrow_of(cw.tile_n);
         tma_load_2d(wb, &tm_w, &wfull[i], cw.kb * (kBlockK / 2), wr, pol_stream);
-        tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], wr, cw.kb * 2, pol_stream);
-        tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], wr, cw.kb * 2, pol_stream);
+        if (!F8) {
+          tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[i], wr, cw.kb * 2, pol_stream);
+          tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[i], wr, cw.kb * 2, pol_stream);
+        }
       }
     }
     griddep_wait();
@@ -631,11 +680,13 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
         if (leader) {
           const int kb = cw.kb, tile_m = cw.tile_m, tile_n = cw.tile_n;
           uint8_t* wb = wring + stage * C::kWStage;
-          mbar_arrive_expect_tx(&wfull[stage], C::kTxW);
+          mbar_arrive_expect_tx(&wfull[stage], kTxW);
           const int wr = wrow_of(tile_n);
           tma_load_2d(wb, &tm_w, &wfull[stage], kb * (kBlockK / 2), wr, pol_stream);
-          tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[stage], wr, kb * 2, pol_stream);
-          tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[stage], wr, kb * 2, pol_stream);
+          if (!F8) {
+            tma_load_2d(wb + C::kWBytes, &tm_s, &wfull[stage], wr, kb * 2, pol_stream);
+            tma_load_2d(wb + C::kWBytes + C::kSABytes, &tm_a, &wfull[stage], wr, kb * 2, pol_stream);
+          }
           mbar_arrive_expect_tx(&xfull[stage], C::kTxX);
           tma_load_2d(xring + stage * C::kXBytes, &tm_x, &xfull[stage], kb * kBlockK, xrow_of(tile_m), pol_keep);
         }
@@ -671,7 +722,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
     if (dual_issue(0) && leader) drain_mmas(drain);
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_i8(BT);
+    constexpr uint32_t idesc = F8 ? idesc_f8(BT) : idesc_i8(BT);
     // A wait costs about as much as a K-block of small MMAs, so the loop waits
     // as little as it can: once for all the preloaded activation tiles; the
     // activation tiles of later blocks are waited for by the expansion warps,
@@ -739,13 +790,14 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
               const uint64_t adesc = smem_desc_k_sw128(smem_u32(aring + slot * (kBlockN * kBlockK)));
 #pragma unroll
               for (int j = 0; j < kBlockK / 32; ++j)
-                mma_i8_ss(tmem_base, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
-                          (kb + r > kb0 || j > 0) ? 1u : 0u);
+                mma_ss_k<F8>(tmem_base, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc,
+                             (kb + r > kb0 || j > 0) ? 1u : 0u);
             } else {
               const uint32_t a_col = tmem_base + C::kAccCols + slot * 32;
 #pragma unroll
               for (int j = 0; j < kBlockK / 32; ++j)
-                mma_i8_ts(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (kb + r > kb0 || j > 0) ? 1u : 0u);
+                mma_ts_k<F8>(tmem_base, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc,
+                             (kb + r > kb0 || j > 0) ? 1u : 0u);
             }
           };
           int r = 0;
@@ -772,7 +824,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
             const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + stage * C::kXBytes));
 #pragma unroll
             for (int j = 0; j < kBlockK / 32; ++j)
-              mma_i8_ss(tmem_base, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, 1u);
+              mma_ss_k<F8>(tmem_base, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, 1u);
           }
         }
         it += run;
@@ -955,27 +1007,38 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
           goto epi_done;
         tc_fence_after();
         const uint8_t* wb = wring + stage * C::kWStage;
-        const uint8_t* ss = wb + C::kWBytes;
-        const uint8_t* sa = ss + C::kSABytes;
-        const uint32_t s0 = ss[r], s1 = ss[kBlockN + r];
-        const uint32_t a0 = (uint32_t)sa[r] * 0x01010101u, a1 = (uint32_t)sa[kBlockN + r] * 0x01010101u;
         const uint32_t wrow = smem_u32(wb) + r * (kBlockK / 2);
         uint32_t v[32];
+        if constexpr (F8) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 q = lds128(wrow + ((c ^ sw) << 4));
-          const uint32_t s = c < 2 ? s0 : s1;
-          const uint32_t a4 = c < 2 ? a0 : a1;
-          if constexpr ((DQ & 1) != 0) {
-            naive_expand_word(q.x, s, a4 & 0xFFu, v[8 * c + 0], v[8 * c + 1]);
-            naive_expand_word(q.y, s, a4 & 0xFFu, v[8 * c + 2], v[8 * c + 3]);
-            naive_expand_word(q.z, s, a4 & 0xFFu, v[8 * c + 4], v[8 * c + 5]);
-            naive_expand_word(q.w, s, a4 & 0xFFu, v[8 * c + 6], v[8 * c + 7]);
-          } else {
-            lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
-            lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
-            lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
-            lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
+          for (int c = 0; c < 4; ++c) {
+            const uint4 q = lds128(wrow + ((c ^ sw) << 4));
+            w4_word_to_e4m3(q.x, v[8 * c + 0], v[8 * c + 1]);
+            w4_word_to_e4m3(q.y, v[8 * c + 2], v[8 * c + 3]);
+            w4_word_to_e4m3(q.z, v[8 * c + 4], v[8 * c + 5]);
+            w4_word_to_e4m3(q.w, v[8 * c + 6], v[8 * c + 7]);
+          }
+        } else {
+          const uint8_t* ss = wb + C::kWBytes;
+          const uint8_t* sa = ss + C::kSABytes;
+          const uint32_t s0 = ss[r], s1 = ss[kBlockN + r];
+          const uint32_t a0 = (uint32_t)sa[r] * 0x01010101u, a1 = (uint32_t)sa[kBlockN + r] * 0x01010101u;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 q = lds128(wrow + ((c ^ sw) << 4));
+            const uint32_t s = c < 2 ? s0 : s1;
+            const uint32_t a4 = c < 2 ? a0 : a1;
+            if constexpr ((DQ & 1) != 0) {
+              naive_expand_word(q.x, s, a4 & 0xFFu, v[8 * c + 0], v[8 * c + 1]);
+              naive_expand_word(q.y, s, a4 & 0xFFu, v[8 * c + 2], v[8 * c + 3]);
+              naive_expand_word(q.z, s, a4 & 0xFFu, v[8 * c + 4], v[8 * c + 5]);
+              naive_expand_word(q.w, s, a4 & 0xFFu, v[8 * c + 6], v[8 * c + 7]);
+            } else {
+              lqq_expand_word(q.x, s, a4, v[8 * c + 0], v[8 * c + 1]);
+              lqq_expand_word(q.y, s, a4, v[8 * c + 2], v[8 * c + 3]);
+              lqq_expand_word(q.z, s, a4, v[8 * c + 4], v[8 * c + 5]);
+              lqq_expand_word(q.w, s, a4, v[8 * c + 6], v[8 * c + 7]);
+            }
           }
         }
         if (to_smem) {
@@ -1056,7 +1119,8 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
         if (!__all_sync(0xffffffffu, mbar_wait(xfirst, 0, abort_flag))) goto epi_done;
       }
       if constexpr (!OUT_I32) {
-        auto sx_at = [&](int m) { return FQ ? sxs[m - m0] : ld_dep(p.s_x + m); };
+        // W4 x FP8: one activation scale for the tensor
+        auto sx_at = [&](int m) { return FQ ? sxs[m - m0] : ld_dep(p.s_x + (F8 ? 0 : m)); };
         if constexpr (CS >= 2) {
 #pragma unroll
           for (int j = 0; j < kSxRegs; ++j) {
@@ -1114,7 +1178,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
               tmem_ld_32x32b_x32(t_lane, w);
               tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] = w[i] + w[16 + i];
+              for (int i = 0; i < 16; ++i) v[i] = acc_add<F8>(w[i], w[16 + i]);
             } else {
               tmem_ld_32x32b_x16(t_lane, v);
               tmem_ld_wait();
@@ -1192,16 +1256,16 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
               for (int sidx = 0; sidx < CS - 1; ++sidx) {
                 if constexpr (T == 2) {
                   const uint2 w2 = *reinterpret_cast<const uint2*>(red + (sidx * kBlockN + r) * 2);
-                  acc[0] += w2.x;
-                  acc[1] += w2.y;
+                  acc[0] = acc_add<F8>(acc[0], w2.x);
+                  acc[1] = acc_add<F8>(acc[1], w2.y);
                 } else {
 #pragma unroll
                   for (int q = 0; q < TCH; q += 4) {
                     const uint4 w4 = *reinterpret_cast<const uint4*>(red + red_off(sidx, (c0 + q) / 4));
-                    acc[q] += w4.x;
-                    acc[q + 1] += w4.y;
-                    acc[q + 2] += w4.z;
-                    acc[q + 3] += w4.w;
+                    acc[q] = acc_add<F8>(acc[q], w4.x);
+                    acc[q + 1] = acc_add<F8>(acc[q + 1], w4.y);
+                    acc[q + 2] = acc_add<F8>(acc[q + 2], w4.z);
+                    acc[q + 3] = acc_add<F8>(acc[q + 3], w4.w);
                   }
                 }
               }
@@ -1219,7 +1283,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
                     if constexpr (OUT_I32) {
                       reinterpret_cast<int32_t*>(p.out)[(size_t)m * p.N + n] = (int32_t)acc[i];
                     } else {
-                      const float y = __fmul_rn(__int2float_rn((int32_t)acc[i]), __fmul_rn(sxm, sc));
+                      const float y = __fmul_rn(acc_f32<F8>(acc[i]), __fmul_rn(sxm, sc));
                       reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)m * p.N + n] = __float2bfloat16_rn(y);
                     }
                   }
@@ -1236,14 +1300,16 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
           for (int cc = 0; cc < BT / CH; ++cc) {
             const float sx_cur = sx_next;
             if (cc + 1 < BT / CH)
-              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < mend) ? ld_dep(p.s_x + m0 + (cc + 1) * CH + lane) : 0.0f;
+              sx_next = (!OUT_I32 && m0 + (cc + 1) * CH + lane < mend)
+                            ? ld_dep(p.s_x + (F8 ? 0 : m0 + (cc + 1) * CH + lane))
+                            : 0.0f;
             uint32_t v[32];
             if (dual) {
               // 16-token tile, two issuers: the sum of accumulator columns [0, 16) and [16, 32)
               tmem_ld_32x32b_x32(t_lane, v);
               tmem_ld_wait();
 #pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] += v[16 + i];
+              for (int i = 0; i < 16; ++i) v[i] = acc_add<F8>(v[i], v[16 + i]);
             } else {
               tmem_load_cols<CH>(t_lane + cc * CH, v);
             }
@@ -1251,7 +1317,7 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
               if constexpr (SWI)
                 store_chunk_swiglu<CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
               else
-                store_chunk<OUT_I32, CH>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
+                store_chunk<OUT_I32, CH, F8>(p, m0 + cc * CH, mend, n, n_ok, v, sx_cur, sc);
             } else {
 #pragma unroll
               for (int i = 0; i < CH; ++i) {
