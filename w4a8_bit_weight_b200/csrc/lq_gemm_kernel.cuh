@@ -582,46 +582,39 @@ __global__ void __launch_bounds__(gemm_threads(EG), GemmCfg<BT, CS, DQ>::kTmemCo
   // The dual-issue form of the MMA loop (see `dual`): issuer i takes the
   // K-blocks b = i, i + 2, ... into accumulator columns [16 i, 16 i + 16).
   // Expansion finishes K-blocks in order, so a completed last block covers
-  // every block before it; each slot is used once (phase 0).  If this
-  // issuer's last block is already expanded when the activations have landed
-  // (the usual case: the weights were streamed and expanded before the
-  // dependency wait), all its MMAs go out as one run; otherwise (a CTA that
-  // started late and is still expanding) each block's MMAs go out as soon as
-  // that block is ready, so that the issue overlaps the rest of the
-  // expansion.  Returns whether this issuer has MMAs in flight (to be drained
-  // before TMEM is freed); the accumulators are committed only if every
-  // block was issued.
+  // every block before it; each slot is used once (phase 0).  Returns whether
+  // this issuer has MMAs in flight (to be drained before TMEM is freed).
   auto dual_issue = [&](int i) -> bool {
-    bool issued = false;
+    bool ok = true;
     if (leader) {
       constexpr uint32_t idesc = F8 ? idesc_f8(BT) : idesc_i8(BT);
-      bool ok = mbar_wait(xfirst, 0, abort_flag);
+      ok = mbar_wait(xfirst, 0, abort_flag);
       const int bl = ((total_u - 1 - i) & 1) ? total_u - 2 : total_u - 1;  // last block of this issuer
-      const bool all_ready =
-          ok && (ovf && bl == A ? mbar_try_wait(smem_u32(ovfull), 0) : mbar_try_wait(smem_u32(&afull[bl]), 0));
-      const uint32_t d = tmem_base + (uint32_t)(16 * i);
-      for (int b = i; b < total_u && ok; b += 2) {
-        if (!all_ready) ok = (ovf && b == A) ? mbar_wait(ovfull, 0, abort_flag) : mbar_wait(&afull[b], 0, abort_flag);
-        if (!ok) break;
-        if (!all_ready || b == i) tc_fence_after();
-        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + b * C::kXBytes));
-        if (ovf && b == A) {
-          // the overflow block: A from the weight stages it was expanded into
-          const uint64_t adesc = smem_desc_k_sw128(smem_u32(wring));
+      if (ok && !(ovf && bl == A ? mbar_try_wait(smem_u32(ovfull), 0) : mbar_try_wait(smem_u32(&afull[bl]), 0)))
+        for (int b = i; b <= bl && ok; b += 2)
+          ok = (ovf && b == A) ? mbar_wait(ovfull, 0, abort_flag) : mbar_wait(&afull[b], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(16 * i);
+        for (int b = i; b < total_u; b += 2) {
+          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xring + b * C::kXBytes));
+          if (ovf && b == A) {
+            // the overflow block: A from the weight stages it was expanded into
+            const uint64_t adesc = smem_desc_k_sw128(smem_u32(wring));
 #pragma unroll
-          for (int j = 0; j < kBlockK / 32; ++j)
-            mma_ss_k<F8>(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
-        } else {
-          const uint32_t a_col = tmem_base + C::kAccCols + b * 32;
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_ss_k<F8>(d, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+          } else {
+            const uint32_t a_col = tmem_base + C::kAccCols + b * 32;
 #pragma unroll
-          for (int j = 0; j < kBlockK / 32; ++j)
-            mma_ts_k<F8>(d, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_ts_k<F8>(d, a_col + j * 8, bdesc + (uint64_t)(2 * j), idesc, (b > i || j > 0) ? 1u : 0u);
+          }
         }
-        issued = true;
+        tc_commit(accfull);
       }
-      if (ok && issued) tc_commit(accfull);
     }
-    return __shfl_sync(0xffffffffu, issued ? 1 : 0, 0) != 0;
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   };
   // waits (bounded) until this thread's issued MMAs have finished
   auto drain_mmas = [&](uint64_t* bar) {
