@@ -256,25 +256,32 @@ def run_ours(args, rank, world, local_rank):
     # lq_w4a8_linear's workspace, for its side measurement (fused vs two launches)
     lin_ws_need = max(lq.lq_w4a8_linear_workspace_size(M, w.N, w.K, lq.LINEAR_TWO_LAUNCHES) for M in Ms)
     ws_lin = torch.zeros(max(lin_ws_need, 16), dtype=torch.uint8, device=dev)
-    # pinned host buffers for the end-to-end variant: the step's batches are the first M
-    # rows of one token set, so one copy of the first max(M) rows brings all of its inputs
+    # pinned host buffers for the end-to-end variant.  The library reads activations from and
+    # writes outputs to pinned host memory directly (zero-copy I/O, lq.h): the step's
+    # quantizers read their rows of X_host over the host link and its GEMMs write their rows
+    # of out_host.  Where the device cannot address them at the same pointer, the variant
+    # copies instead: the step's batches are the first M rows of one token set, so one copy
+    # of the first max(M) rows brings all of its inputs, and one copy takes all outputs back.
     X_host = X.pin_memory()
     out_host = torch.empty(sum(Ms), w.N, dtype=torch.bfloat16).pin_memory()
-    Xd_e2e = torch.empty_like(Xd)
+    out_host_buf = {M: out_host[out_off[M]:out_off[M] + M] for M in Ms}
+    zero_copy = lq.lq_device_addressable(X_host) and lq.lq_device_addressable(out_host)
+    Xd_e2e = None if zero_copy else torch.empty_like(Xd)
 
     stream = torch.cuda.Stream(dev)
     counter = [0]
 
     def step(e2e=False):
-        if e2e:
+        if e2e and not zero_copy:
             Xd_e2e[:Mx].copy_(X_host[:Mx], non_blocking=True)
         for M in Ms:
-            src = Xd_e2e[:M] if e2e else Xd[:M]
+            src = (X_host[:M] if zero_copy else Xd_e2e[:M]) if e2e else Xd[:M]
             lq.lq_quantize_act(src, out=(xq_buf[M], sx_buf[M]))
             wq = sets[counter[0] % n_sets]
             counter[0] += 1
-            lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=out_buf[M], workspace_buf=ws)
-        if e2e:
+            dst = out_host_buf[M] if (e2e and zero_copy) else out_buf[M]
+            lq.lq_w4a8_gemm(xq_buf[M], sx_buf[M], *wq, out=dst, workspace_buf=ws)
+        if e2e and not zero_copy:
             out_host.copy_(out_all, non_blocking=True)
 
     def capture(nsteps, e2e=False):
@@ -417,14 +424,18 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if ms_e2e is not None:
-        h2d = max(Ms) * w.K * 2
+        h2d = (sum(Ms) if zero_copy else max(Ms)) * w.K * 2
         d2h = sum(Ms) * w.N * 2
         res["e2e"] = {"value": world * step_bytes * K_ / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": ms_e2e / K_,
-                      "how": "per step: one pinned host -> device copy of the activation rows (every "
-                             "batch of the step is a prefix of them), quantize_act + gemm per M, one device -> "
-                             "pinned host copy of all outputs; same CUDA graph method"}
+                      "how": ("per step and M: lq_quantize_act reads the batch's bf16 rows from pinned host "
+                              "memory and lq_w4a8_gemm writes its bf16 outputs to pinned host memory, both "
+                              "directly over the host link (zero-copy I/O); same CUDA graph method"
+                              if zero_copy else
+                              "per step: one pinned host -> device copy of the activation rows (every "
+                              "batch of the step is a prefix of them), quantize_act + gemm per M, one device -> "
+                              "pinned host copy of all outputs; same CUDA graph method")}
     if lin_us:
         res["linear"] = {
             "what": "lq_w4a8_linear (activation quantization + GEMM) per M, one fused launch vs the "

@@ -14,6 +14,17 @@
  * Conventions for every entry point
  *   - All pointers are DEVICE pointers unless stated otherwise.  The caller
  *     owns every buffer; the library never allocates or frees device memory.
+ *   - Exception (zero-copy I/O): the bf16 activations X that a call reads
+ *     (lq_quantize_act, lq_quantize_act_f8, lq_w4a8_linear*) and the outputs
+ *     that a GEMM writes (`out` of every GEMM entry point) may also be host
+ *     memory that the current device addresses at the same pointer: pinned
+ *     with cudaHostAlloc, or registered with cudaHostRegister as mapped.  The
+ *     kernels then read or write it over the host link directly, with no
+ *     copy (for decode batches this is faster than a copy before and after:
+ *     copy-engine transfers also end the programmatic-launch chain).  Any
+ *     other host memory (pageable, or mapped at a different address) is
+ *     refused with LQ_ERR_INVALID_ARG before anything is launched.  Weights,
+ *     scales, int8 activations and workspaces must be device memory.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  All work is enqueued asynchronously on it; nothing blocks the
  *     host except lq_get_device_error.
@@ -406,6 +417,13 @@ LQ_API lq_status lq_quantize_weights_w4(const void* W_bf16, int N, int K, uint8_
 LQ_API lq_status lq_quantize_act_f8(const void* X_bf16, int M, int K, uint8_t* x_f8, float* s_x, void* stream);
 LQ_API lq_status lq_w4f8_gemm(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4, const float* s_w,
                               void* out_bf16, int M, int N, int K, void* stream);
+
+/*
+ * lq_device_addressable -- 1 if the current device can read and write `p`
+ *   at that address (device or managed memory, or host memory mapped at the
+ *   same address: the zero-copy rule above), else 0.  Launches nothing.
+ */
+LQ_API int lq_device_addressable(const void* p);
 
 /*
  * lq_test_wait_timeout -- TEST ONLY: launches a one-CTA kernel whose first

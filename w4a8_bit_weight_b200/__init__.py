@@ -60,6 +60,7 @@ def load_library(path: str = LIB_PATH):
         P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         sig = {
             "lq_version": ([], I),
+            "lq_device_addressable": ([P], I),
             "lq_status_string": ([I], ctypes.c_char_p),
             "lq_quantize_weights": ([P, I, I, I, P, P, P, P, P], I),
             "lq_quantize_act": ([P, I, I, P, P, P], I),
@@ -125,6 +126,30 @@ def _need(t: torch.Tensor, dtype, name: str, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _need_io(t: torch.Tensor, dtype, name: str, shape=None):
+    """_need, except that a pinned host tensor is accepted too: activations read and
+    outputs written by the kernels directly over the host link (zero-copy I/O, lq.h)."""
+    if isinstance(t, torch.Tensor) and not t.is_cuda and t.is_pinned():
+        if t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+        return
+    _need(t, dtype, name, shape)
+
+
+def _cuda_device(t: torch.Tensor) -> torch.device:
+    """The device a call runs on: the tensor's, or the current one for a pinned host tensor."""
+    return t.device if t.is_cuda else torch.device("cuda", torch.cuda.current_device())
+
+
+def lq_device_addressable(t: torch.Tensor) -> bool:
+    """Whether the current device reads and writes t's memory at its address (lq.h)."""
+    return bool(load_library().lq_device_addressable(_ptr(t)))
+
+
 # ----------------------------------------------------------------------------
 # workspace: one zero-filled scratch buffer per device, grown on demand.  The
 # kernels leave it zero-filled after every call, so it is cleared only once.
@@ -173,16 +198,18 @@ def lq_quantize_weights(W: torch.Tensor, group: int = GROUP, out=None):
 
 
 def lq_quantize_act(X: torch.Tensor, out=None):
-    """Per-token symmetric INT8 of X [M, K] bf16 -> (x_q [M,K] int8, s_x [M] f32)."""
+    """Per-token symmetric INT8 of X [M, K] bf16 -> (x_q [M,K] int8, s_x [M] f32).
+    X may be a pinned host tensor (read over the host link)."""
     lib = load_library()
-    _need(X, torch.bfloat16, "X")
+    _need_io(X, torch.bfloat16, "X")
     M, K = X.shape
+    dev = _cuda_device(X)
     if out is None:
-        out = (torch.empty(M, K, dtype=torch.int8, device=X.device),
-               torch.empty(M, dtype=torch.float32, device=X.device))
+        out = (torch.empty(M, K, dtype=torch.int8, device=dev),
+               torch.empty(M, dtype=torch.float32, device=dev))
     xq, sx = out
-    with torch.cuda.device(X.device):
-        _check("lq_quantize_act", lib.lq_quantize_act(_ptr(X), M, K, _ptr(xq), _ptr(sx), _stream(X.device)))
+    with torch.cuda.device(dev):
+        _check("lq_quantize_act", lib.lq_quantize_act(_ptr(X), M, K, _ptr(xq), _ptr(sx), _stream(dev)))
     return xq, sx
 
 
@@ -220,7 +247,7 @@ def _gemm(x_q, s_x, qw, s_u8, a_u8, s_c, out, group, block_t, split_k, grid, out
     odt = torch.int32 if out_i32 else torch.bfloat16
     if out is None:
         out = torch.empty(M, N, dtype=odt, device=x_q.device)
-    _need(out, odt, "out", (M, N))
+    _need_io(out, odt, "out", (M, N))
     with torch.cuda.device(x_q.device):
         sch = _sched(schedule, split_k, grid)
         need = lq_w4a8_gemm_workspace_size(M, N, K, block_t, split_k, grid, sch)
@@ -269,7 +296,7 @@ def lq_w4a8_gemm_swiglu(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = GR
         raise ValueError("the gate/up weights come in row pairs")
     if out is None:
         out = torch.empty(M, N // 2, dtype=torch.bfloat16, device=x_q.device)
-    _need(out, torch.bfloat16, "out", (M, N // 2))
+    _need_io(out, torch.bfloat16, "out", (M, N // 2))
     with torch.cuda.device(x_q.device):
         ws = workspace_buf
         sch = _sched(schedule, split_k, 0)
@@ -297,24 +324,25 @@ def lq_w4a8_linear(X, qw, s_u8, a_u8, s_c, out=None, group: int = GROUP, workspa
     small decode batches, two launches otherwise (lq_w4a8_linear in lq.h); `path`
     forces one of them (LINEAR_*)."""
     lib = load_library()
-    _need(X, torch.bfloat16, "X")
+    _need_io(X, torch.bfloat16, "X")
     M, K = X.shape
     N = qw.shape[0]
     _need(qw, torch.uint8, "qw", (N, K // 2))
     _need(s_u8, torch.uint8, "s_u8", (K // group, N))
     _need(a_u8, torch.uint8, "a_u8", (K // group, N))
     _need(s_c, torch.float32, "s_c", (N,))
+    dev = qw.device
     if out is None:
-        out = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
-    _need(out, torch.bfloat16, "out", (M, N))
-    with torch.cuda.device(X.device):
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    _need_io(out, torch.bfloat16, "out", (M, N))
+    with torch.cuda.device(dev):
         ws = workspace_buf
         if ws is None:
-            ws = workspace(lq_w4a8_linear_workspace_size(M, N, K, path), X.device, kind="linear")
+            ws = workspace(lq_w4a8_linear_workspace_size(M, N, K, path), dev, kind="linear")
         nbytes = ws.numel() * ws.element_size() if ws is not None else 0
         _check("lq_w4a8_linear", lib.lq_w4a8_linear_ex(
             _ptr(X), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out), M, N, K, group,
-            _ptr(ws), nbytes, path, _stream(X.device)))
+            _ptr(ws), nbytes, path, _stream(dev)))
     return out
 
 
@@ -333,7 +361,7 @@ def lq_w4a8_gemm_noalloc(x_q, s_x, qw, s_u8, a_u8, s_c, out=None, group: int = G
     _need(s_c, torch.float32, "s_c", (N,))
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x_q.device)
-    _need(out, torch.bfloat16, "out", (M, N))
+    _need_io(out, torch.bfloat16, "out", (M, N))
     with torch.cuda.device(x_q.device):
         _check("lq_w4a8_gemm_noalloc", lib.lq_w4a8_gemm_noalloc(
             _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out),
@@ -363,7 +391,7 @@ def lq_w4a8_grouped_gemm(x_q, s_x, qw, s_u8, a_u8, s_c, m_off, N: int, out=None,
     odt = torch.int32 if out_i32 else torch.bfloat16
     if out is None:
         out = torch.empty(M, N, dtype=odt, device=x_q.device)
-    _need(out, odt, "out", (M, N))
+    _need_io(out, odt, "out", (M, N))
     with torch.cuda.device(x_q.device):
         _check("lq_w4a8_grouped_gemm", lib.lq_w4a8_grouped_gemm_ex(
             _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(m_off), G, _ptr(out),
@@ -390,7 +418,7 @@ def lq_w4a8_gemm_ablation(x_q, s_x, qw, s_u8, a_u8, s_c, variant: int, block_t: 
     odt = torch.int32 if out_i32 else torch.bfloat16
     if out is None:
         out = torch.empty(M, N, dtype=odt, device=x_q.device)
-    _need(out, odt, "out", (M, N))
+    _need_io(out, odt, "out", (M, N))
     with torch.cuda.device(x_q.device):
         _check("lq_w4a8_gemm_ablation", lib.lq_w4a8_gemm_ablation(
             _ptr(x_q), _ptr(s_x), _ptr(qw), _ptr(s_u8), _ptr(a_u8), _ptr(s_c), _ptr(out), M, N, K, group,
@@ -429,13 +457,14 @@ def lq_quantize_weights_w4(W: torch.Tensor, out=None):
 def lq_quantize_act_f8(X: torch.Tensor, out=None):
     """W4 x FP8 variant: e4m3 codes with one scale for the tensor -> (x_f8 [M, K] uint8, s_x [1] fp32)."""
     lib = load_library()
-    _need(X, torch.bfloat16, "X")
+    _need_io(X, torch.bfloat16, "X")
     M, K = X.shape
-    x_f8, s_x = out if out is not None else (torch.empty(M, K, dtype=torch.uint8, device=X.device),
-                                             torch.empty(1, dtype=torch.float32, device=X.device))
-    with torch.cuda.device(X.device):
+    dev = _cuda_device(X)
+    x_f8, s_x = out if out is not None else (torch.empty(M, K, dtype=torch.uint8, device=dev),
+                                             torch.empty(1, dtype=torch.float32, device=dev))
+    with torch.cuda.device(dev):
         _check("lq_quantize_act_f8", lib.lq_quantize_act_f8(_ptr(X), M, K, _ptr(x_f8), _ptr(s_x),
-                                                            _stream(X.device)))
+                                                            _stream(dev)))
     return x_f8, s_x
 
 
@@ -450,7 +479,7 @@ def lq_w4f8_gemm(x_f8, s_x, qw4, s_w, out=None):
     _need(s_w, torch.float32, "s_w", (N,))
     if out is None:
         out = torch.empty(M, N, dtype=torch.bfloat16, device=x_f8.device)
-    _need(out, torch.bfloat16, "out", (M, N))
+    _need_io(out, torch.bfloat16, "out", (M, N))
     with torch.cuda.device(x_f8.device):
         _check("lq_w4f8_gemm", lib.lq_w4f8_gemm(_ptr(x_f8), _ptr(s_x), _ptr(qw4), _ptr(s_w), _ptr(out), M, N, K,
                                                 _stream(x_f8.device)))

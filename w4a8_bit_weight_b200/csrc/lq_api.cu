@@ -57,6 +57,30 @@ lq_status current_device(DeviceInfo** out) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The bf16 activations a call reads and the outputs it writes may be host
+// memory that the current device addresses directly (pinned with
+// cudaHostAlloc, or registered with cudaHostRegister as mapped): the kernels
+// then read or write it over the host link, with no copy.  Device and managed
+// memory are addressable too.  Memory that CUDA does not know (pageable host
+// memory) or host memory mapped at another address is refused before any
+// launch.
+bool device_addressable(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  switch (a.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+      return true;
+    case cudaMemoryTypeHost:
+      return a.devicePointer == p;
+    default:
+      return false;
+  }
+}
+
 // ------------------------------------------------------------ tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -470,6 +494,7 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
+  if (!device_addressable(out)) return LQ_ERR_INVALID_ARG;
   Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms);
   if (swiglu) {
     // the SwiGLU epilogue runs on the tile kernel's cluster schedules and the
@@ -598,6 +623,7 @@ lq_status lq_w4a8_linear_ex(const void* X_bf16, const uint8_t* qw, const uint8_t
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
+  if (!device_addressable(X_bf16) || !device_addressable(out_bf16)) return LQ_ERR_INVALID_ARG;
   const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, dev->sms);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (path == LQ_LINEAR_FUSED && !fused_eligible(s, M)) return LQ_ERR_UNSUPPORTED_SHAPE;
@@ -649,6 +675,12 @@ extern "C" {
 
 int lq_version(void) { return 100; }
 
+int lq_device_addressable(const void* p) {
+  DeviceInfo* dev = nullptr;
+  if (p == nullptr || current_device(&dev) != LQ_OK) return 0;
+  return device_addressable(p) ? 1 : 0;
+}
+
 const char* lq_status_string(lq_status status) {
   switch (status) {
     case LQ_OK: return "LQ_OK";
@@ -686,6 +718,7 @@ lq_status lq_quantize_act(const void* X_bf16, int M, int K, int8_t* x_q, float* 
   DeviceInfo* dev = nullptr;
   lq_status st = current_device(&dev);
   if (st != LQ_OK) return st;
+  if (!device_addressable(X_bf16)) return LQ_ERR_INVALID_ARG;
   return launch_ex(lq::quantize_act_kernel, M, lq::kQuantActThreads, 0, 1, pdl_enabled(),
                    static_cast<cudaStream_t>(stream), static_cast<const uint16_t*>(X_bf16), K, x_q, s_x);
 }
@@ -915,6 +948,7 @@ lq_status grouped_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, c
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
+  if (!device_addressable(out)) return LQ_ERR_INVALID_ARG;
   const long long tm_bound = std::min<long long>(((long long)M + (long long)groups * (bt - 1)) / bt, M);
   if (tm_bound * bt > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
   const Schedule s = pair ? make_schedule((int)(tm_bound * bt), N, K, 0, kSchedPair, 0, 0, dev->sms)
@@ -1072,6 +1106,7 @@ lq_status lq_quantize_act_f8(const void* X_bf16, int M, int K, uint8_t* x_f8, fl
   DeviceInfo* dev = nullptr;
   const lq_status st = current_device(&dev);
   if (st != LQ_OK) return st;
+  if (M > 0 && !device_addressable(X_bf16)) return LQ_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // the tensor's amax in s_x's word, the codes, then s_x itself (an empty tensor gets s_x = 1)
   if (cudaMemsetAsync(s_x, 0, sizeof(float), cs) != cudaSuccess) return LQ_ERR_CUDA;
@@ -1096,6 +1131,7 @@ lq_status lq_w4f8_gemm(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
+  if (!device_addressable(out_bf16)) return LQ_ERR_INVALID_ARG;
   return w4f8_impl(x_f8, s_x, qw4, s_w, out_bf16, M, N, K, dev->sms, static_cast<cudaStream_t>(stream));
 }
 
