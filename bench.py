@@ -19,6 +19,14 @@ roofline's denominator) comes from a second graph of K back-to-back GEMM calls
 per M, timed the same way: the launches overlap through programmatic dependent
 launch exactly as in the step, and replay time / K is the time per launch.
 
+The end-to-end variant (`e2e`) runs the same step through the same calls
+with host buffers: each batch's bf16 rows are read from pinned host memory by
+the activation quantizer and each GEMM writes its outputs to pinned host
+memory, both directly over the host link (zero-copy I/O of the library), so
+the transfers sit inside the timed region without copy nodes that would end
+the programmatic-launch chain.  Where the device cannot address the pinned
+buffers, it copies instead (one copy in, one copy out per step).
+
 The default (decode) run also measures, in the same process: the prefill
 layer, a dense INT8 ceiling (torch._int_mm at 8192^3), the MLP up/gate layer
 and the down-projection sweep (every M of both), the fused SwiGLU gate/up pair

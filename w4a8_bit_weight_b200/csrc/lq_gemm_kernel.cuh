@@ -96,9 +96,10 @@ struct GemmCfg {
   static_assert(BT == 16 || BT == 32 || BT == 64 || BT == 128 || BT == 256, "tokens per tile");
   static_assert(CS >= 0 && CS <= 8, "cluster size");
   // shared-memory stages: a ring of activation tiles and a ring of weight tiles
-  // (32-token tiles in 8-CTA clusters keep to 7, so that two CTAs fit an SM)
+  // (32-token tiles in 8-CTA clusters keep to 7, so that two CTAs fit an SM;
+  // 128-token tiles in clusters keep to 7 beside the split-K receive buffer)
   static constexpr int kStages =
-      BT <= 32 ? (BT == 32 && CS == 8 ? 7 : 8) : BT == 64 ? 6 : (BT == 128 ? (CS >= 2 ? 6 : 8) : 5);
+      BT <= 32 ? (BT == 32 && CS == 8 ? 7 : 8) : BT == 64 ? 6 : (BT == 128 ? (CS >= 2 ? 7 : 8) : 5);
   static constexpr int kXBytes = BT * kBlockK;             // int8 activation tile, 128-byte rows (SW128)
   static constexpr int kWBytes = kBlockN * kBlockK / 2;    // packed u4 weight tile, 64-byte rows (SW64)
   static constexpr int kSABytes = 2 * kBlockN;             // 2 groups x 128 rows of u8
