@@ -97,6 +97,8 @@ def _load():
     lib.lq_oracle_f32_to_e4m3.restype = ctypes.c_uint8
     lib.lq_oracle_num_threads.argtypes = []
     lib.lq_oracle_num_threads.restype = I
+    lib.lq_oracle_set_num_threads.argtypes = [I]
+    lib.lq_oracle_set_num_threads.restype = None
     _lib = lib
     return lib
 
@@ -119,6 +121,11 @@ def _u16(a) -> np.ndarray:
 
 def num_threads() -> int:
     return _load().lq_oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops from now on (for a single-core timing)."""
+    _load().lq_oracle_set_num_threads(int(n))
 
 
 def f32_to_bf16(x: float) -> int:

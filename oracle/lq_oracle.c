@@ -79,6 +79,16 @@ int lq_oracle_num_threads(void) {
 #endif
 }
 
+/* Threads the parallel loops use from now on (n >= 1); for timing the oracle
+   on one core beside all of them. */
+void lq_oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ---------------------------------------------------------------------- */
 /* LiquidQuant level 1: per-channel symmetric INT8 in the protective range  */
 /* [-119, 119] (review page: referee summary and circularity rationale,     */
