@@ -183,13 +183,15 @@ def _plan(lib, M, N, K, sms=148, bt=0, sched=0, split=0, grid=0):
 @pytest.mark.parametrize("M,N,K,plan", [
     # (kind, token tile, CTAs per cluster, grid) on 148 SMs; kinds: 1 tiles, 2 persistent, 4 CTA pairs
     (16, 4096, 4096, (1, 16, 4, 128)),       # decode: 4-CTA clusters, one wave
-    (1, 4096, 14336, (1, 16, 8, 256)),       # long K-slices: 8-CTA clusters, two CTAs per SM
+    (1, 4096, 14336, (1, 32, 8, 256)),       # long K-slices: 8-CTA clusters, two CTAs per SM, as 32-token tiles
+    (16, 4096, 14336, (1, 32, 8, 256)),      # the same at 16 tokens
     (32, 4096, 14336, (1, 32, 8, 256)),      # 32-token tiles in 8-CTA clusters fit two per SM (7 stages)
     (64, 4096, 14336, (1, 64, 4, 128)),      # 64-token tiles: 4-CTA clusters, one per SM
     (128, 4096, 14336, (1, 128, 4, 128)),    # 128-token tiles in 4-CTA clusters
     (256, 4096, 14336, (1, 128, 2, 128)),    # 16 pair tiles: too few for pairs; 64 tiles, 2-CTA clusters
     (16, 14336, 4096, (1, 16, 2, 224)),      # 112 tiles: 2-CTA clusters, two per SM
-    (128, 14336, 4096, (1, 128, 1, 112)),    # at most 128 tokens: never pairs
+    (128, 14336, 4096, (2, 128, 1, 112)),    # at most 128 tokens: never pairs; 112 tiles: persistent
+    (512, 4096, 14336, (2, 128, 1, 128)),    # 16 pair tiles: too few; 128 tiles cannot split K: persistent
     (256, 14336, 4096, (4, 256, 2, 112)),    # 56 pair tiles >= 148 / 4: CTA pairs
     (1024, 4096, 14336, (4, 256, 2, 128)),   # 64 pair tiles: 64 pairs
     (4096, 4096, 4096, (4, 256, 2, 148)),    # prefill: 74 persistent pairs
