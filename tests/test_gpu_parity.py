@@ -110,6 +110,8 @@ SHAPES = [
     (16, 256, 512, 0, None, 0, 0),        # the tiny workload
     (1, 256, 512, 0, None, 0, 0),
     (1, 16, 128, 0, None, 0, 0),          # one K-block, N smaller than a tile
+    (8, 4096, 14336, 0, None, 0, 0),      # automatic: 8-CTA clusters with streaming K-slices, 32-token tiles
+    (512, 4096, 1024, 0, None, 0, 0),     # automatic: 128 tiles of 128 x 128 that cannot split K, persistent
     (3, 272, 384, 16, T, 0, 0),           # ragged N (one full + one 16-row tile)
     (17, 384, 1024, 32, T, 0, 0),         # ragged M
     (16, 256, 1024, 16, T, 1, 0),         # one CTA per tile: direct epilogue
