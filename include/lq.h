@@ -311,13 +311,38 @@ LQ_API lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const
 
 /*
  * lq_plan_gemm -- TEST ONLY, touches no device: the schedule lq_w4a8_gemm_ex
- * would run for these arguments on a GPU with `sms` multiprocessors.  On
- * LQ_OK, plan[0..3] = schedule kind (LQ_SCHED_*), token-tile width, CTAs per
- * cluster (0 for stream-K, 2 for CTA pairs), grid size.  Argument errors as
- * in lq_w4a8_gemm_ex (M >= 1 here).
+ * would run for these arguments on a GPU with `sms` multiprocessors, all of
+ * them reachable by clusters of every size (lq_plan_gemm_ex with
+ * cluster_ctas = NULL).  On LQ_OK, plan[0..3] = schedule kind (LQ_SCHED_*),
+ * token-tile width, CTAs per cluster (0 for stream-K, 2 for CTA pairs), grid
+ * size.  Argument errors as in lq_w4a8_gemm_ex (M >= 1 here).
  */
 LQ_API lq_status lq_plan_gemm(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms,
                               int* plan);
+
+/*
+ * lq_plan_gemm_ex -- TEST ONLY, touches no device: lq_plan_gemm on a GPU
+ * whose clusters of 2, 4 and 8 CTAs, two CTAs per SM, place at most
+ * cluster_ctas[0], [1] and [2] CTAs at once (host array of 3 ints, each >= 1,
+ * else LQ_ERR_INVALID_ARG; NULL: 2 x sms each).  The automatic schedule gives
+ * streaming K-slices the widest split whose CTAs fit one wave of that
+ * placement.  lq_device_cluster_ctas gives the current device's numbers, which
+ * lq_w4a8_gemm_ex and the other GEMM calls use.
+ */
+LQ_API lq_status lq_plan_gemm_ex(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms,
+                                 const int* cluster_ctas, int* plan);
+
+/*
+ * lq_device_cluster_ctas -- how many CTAs of 2-, 4- and 8-CTA clusters the
+ * current device holds at once with two CTAs per SM (cluster_ctas: host array
+ * of 3 ints, written on LQ_OK).  A cluster's CTAs share one GPC, so slots
+ * beyond a GPC's last whole cluster stay empty (B200, 148 SMs: 296, 284, 264).
+ * The numbers come from the CUDA occupancy calculator at the first call of
+ * any entry point on the device (2 x SMs where it cannot answer); no kernel
+ * is launched.  LQ_ERR_INVALID_ARG for a NULL array, LQ_ERR_CUDA without a
+ * device, LQ_ERR_ARCH on a device other than sm_100.
+ */
+LQ_API lq_status lq_device_cluster_ctas(int* cluster_ctas);
 
 /*
  * lq_w4a8_gemm_ablation -- TEST AND MEASUREMENT ONLY: the pages' ablation of

@@ -202,6 +202,40 @@ def test_automatic_schedule(lib, M, N, K, plan):
     assert st == 0 and got == plan, got
 
 
+B200_CLUSTER_CTAS = (296, 284, 264)  # 2-, 4-, 8-CTA clusters, two CTAs per SM, on a 148-SM B200
+
+
+def _plan_ex(lib, M, N, K, cl, sms=148):
+    out = (ctypes.c_int * 4)()
+    arr = None if cl is None else (ctypes.c_int * 3)(*cl)
+    st = lib.lq_plan_gemm_ex(M, N, K, 0, 0, 0, 0, sms, arr, out)
+    return st, tuple(out)
+
+
+@pytest.mark.parametrize("M,N,K,flat,placed", [
+    # 34 and 36 weight tiles: 8-CTA clusters would take 272 / 288 CTAs, more than the 264
+    # that B200 places at once, so the placed plan keeps 16-token tiles in 4-CTA clusters
+    (16, 4352, 14336, (1, 32, 8, 272), (1, 16, 4, 136)),
+    (1, 4608, 14336, (1, 32, 8, 288), (1, 16, 4, 144)),
+    # 32 tiles x 8 = 256 CTAs fit one wave either way
+    (16, 4096, 14336, (1, 32, 8, 256), (1, 32, 8, 256)),
+    (16, 3584, 14336, (1, 32, 8, 224), (1, 32, 8, 224)),
+    # 2-CTA clusters reach every SM; 4-CTA decode clusters are one CTA per SM anyway
+    (16, 14336, 4096, (1, 16, 2, 224), (1, 16, 2, 224)),
+    (16, 4096, 4096, (1, 16, 4, 128), (1, 16, 4, 128)),
+])
+def test_schedule_counts_cluster_placement(lib, M, N, K, flat, placed):
+    assert _plan_ex(lib, M, N, K, None) == (0, flat)
+    assert _plan(lib, M, N, K) == (0, flat)  # lq_plan_gemm: every SM reachable
+    assert _plan_ex(lib, M, N, K, B200_CLUSTER_CTAS) == (0, placed)
+
+
+def test_plan_ex_rejects_bad_cluster_table(lib):
+    assert _plan_ex(lib, 16, 4096, 4096, (296, 0, 264))[0] == 1
+    assert _plan_ex(lib, 16, 4096, 4096, (296, 284, -1))[0] == 1
+    assert lib.lq_device_cluster_ctas(None) == 1
+
+
 def test_plan_follows_explicit_choices(lib):
     assert _plan(lib, 16, 256, 1024, bt=16, sched=1, split=2) == (0, (1, 16, 2, 4))
     assert _plan(lib, 16, 256, 1024, bt=16, sched=3, grid=3) == (0, (3, 16, 0, 3))

@@ -112,6 +112,8 @@ SHAPES = [
     (1, 16, 128, 0, None, 0, 0),          # one K-block, N smaller than a tile
     (8, 4096, 14336, 0, None, 0, 0),      # automatic: 8-CTA clusters with streaming K-slices, 32-token tiles
     (512, 4096, 1024, 0, None, 0, 0),     # automatic: 128 tiles of 128 x 128 that cannot split K, persistent
+    (16, 4352, 14336, 0, None, 0, 0),     # automatic: 34 tiles, more 8-CTA clusters than B200 places at once
+    (1, 4608, 14336, 0, None, 0, 0),      # automatic: the same with 36 tiles at one token
     (3, 272, 384, 16, T, 0, 0),           # ragged N (one full + one 16-row tile)
     (17, 384, 1024, 32, T, 0, 0),         # ragged M
     (16, 256, 1024, 16, T, 1, 0),         # one CTA per tile: direct epilogue
@@ -284,3 +286,22 @@ def test_workload_mlp_up():
 
 def test_workload_down_sweep():
     _workload_check("down_sweep", synth.WORKLOADS["down_sweep"].Ms)
+
+
+def test_device_cluster_table_and_the_schedule_it_gives():
+    """The device's cluster placement (lq_device_cluster_ctas) and the automatic
+    schedule's use of it: a split's CTAs fit one wave of the clusters it needs."""
+    import ctypes
+    torch.cuda.set_device(0)
+    lib = lq.load_library()
+    cl = (ctypes.c_int * 3)()
+    assert lib.lq_device_cluster_ctas(cl) == 0
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for i, c in enumerate((2, 4, 8)):
+        assert 0 < cl[i] <= 2 * sms and cl[i] % c == 0, tuple(cl)
+    plan = (ctypes.c_int * 4)()
+    for (M, N, K) in ((16, 4352, 14336), (1, 4608, 14336), (16, 4096, 14336), (16, 14336, 4096)):
+        assert lib.lq_plan_gemm_ex(M, N, K, 0, 0, 0, 0, sms, cl, plan) == 0
+        kind, bt, cs, grid = tuple(plan)
+        if kind == 1 and cs in (2, 4, 8) and grid > sms:  # two CTAs per SM: the clusters must all fit
+            assert grid <= cl[(2, 4, 8).index(cs)], (M, N, K, tuple(plan), tuple(cl))

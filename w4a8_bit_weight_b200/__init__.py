@@ -82,6 +82,8 @@ def load_library(path: str = LIB_PATH):
             "lq_w4a8_gemm_ablation": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P], I),
             "lq_test_wait_timeout": ([P], I),
             "lq_plan_gemm": ([I, I, I, I, I, I, I, I, P], I),
+            "lq_plan_gemm_ex": ([I, I, I, I, I, I, I, I, P, P], I),
+            "lq_device_cluster_ctas": ([P], I),
             "lq_quantize_weights_w4": ([P, I, I, P, P, P], I),
             "lq_quantize_act_f8": ([P, I, I, P, P, P], I),
             "lq_w4f8_gemm": ([P, P, P, P, P, I, I, I, P], I),

@@ -30,9 +30,43 @@ struct DeviceInfo {
   std::atomic<bool> ready{false};
   bool sm100 = false;
   int sms = 0;
+  int cluster_ctas[3] = {0, 0, 0};  // see cluster_fit
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
+
+// An empty kernel that only the occupancy query below names (never launched).
+__global__ void cluster_fit_probe_kernel() {}
+
+// How many CTAs of c-CTA clusters the device holds at once when two CTAs share
+// an SM.  A cluster's CTAs must sit in one GPC, so a GPC's slots beyond its
+// last whole cluster stay empty: on B200 (148 SMs, 296 slots) clusters of 2, 4
+// and 8 place 296, 284 and 264 CTAs.  The occupancy calculator answers for an
+// empty 192-thread kernel whose shared memory admits exactly two CTAs per SM
+// (as the tile kernel's does wherever two of its CTAs share an SM); if it
+// cannot answer, 2 x sms.
+int cluster_fit(int c, int sms) {
+  constexpr int kSmem = 100 * 1024;  // two fit in an SM's 228 KB, three do not
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kSmem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = c;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&n, cluster_fit_probe_kernel, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    return 2 * sms;
+  }
+  return std::min(2 * sms, n * c);
+}
 
 lq_status current_device(DeviceInfo** out) {
   int dev = 0;
@@ -48,6 +82,8 @@ lq_status current_device(DeviceInfo** out) {
         return LQ_ERR_CUDA;
       d.sm100 = (major == 10 && minor == 0);
       d.sms = sms;
+      if (d.sm100)
+        for (int i = 0; i < 3; ++i) d.cluster_ctas[i] = cluster_fit(2 << i, sms);
       d.ready.store(true, std::memory_order_release);
     }
   }
@@ -214,7 +250,15 @@ bool fits_two_per_sm(int bt, int cs) {
   return false;
 }
 
-Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms) {
+// CTAs of c-CTA clusters that fit at once, two per SM: from the device's table
+// (cluster_fit) where there is one, else every SM counted
+long long cluster_slots(int c, int sms, const int* cl) {
+  const int i = c == 2 ? 0 : c == 4 ? 1 : c == 8 ? 2 : -1;
+  return (cl != nullptr && i >= 0 && cl[i] > 0) ? std::min<long long>(cl[i], 2LL * sms) : 2LL * sms;
+}
+
+Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms,
+                       const int* cl) {
   Schedule s;
   int kind = schedule;
   int bt = block_t ? block_t : auto_block_t(M);
@@ -294,10 +338,14 @@ Schedule make_schedule(int M, int N, int K, int block_t, int schedule, int split
       }
     // When a CTA's K-slice is longer than its preloaded stages, the ring
     // streams the rest anyway and more CTAs stream faster: where two CTAs of
-    // a wider split fit one SM, use that capacity.
+    // a wider split fit one SM, use that capacity -- as far as the device can
+    // place clusters of that size.  One cluster more than fit starts a second
+    // wave (measured on B200 at 16 x 4352 x 14336: 272 CTAs in 8-CTA
+    // clusters, 18.3 us; 136 in 4-CTA clusters, 16.3 us; 16 x 4096 x 14336,
+    // 256 CTAs in one wave, 11.5 us).
     if (s.KB / cs > stages_of(s.bt) && s.bt <= 64)
       for (int c = max_split(s.bt); c > cs; c /= 2)
-        if (fits_two_per_sm(s.bt, c) && s.tiles * c <= 2LL * sms && s.KB / c >= 4) {
+        if (fits_two_per_sm(s.bt, c) && s.tiles * c <= cluster_slots(c, sms, cl) && s.KB / c >= 4) {
           cs = c;
           break;
         }
@@ -504,13 +552,14 @@ lq_status gemm_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, cons
   st = current_device(&dev);
   if (st != LQ_OK) return st;
   if (!device_addressable(out)) return LQ_ERR_INVALID_ARG;
-  Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms);
+  Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, dev->sms, dev->cluster_ctas);
   if (swiglu) {
     // the SwiGLU epilogue runs on the tile kernel's cluster schedules and the
     // CTA-pair kernel: a persistent choice becomes one cluster per tile
     if (s.kind == kSchedStreamK || (s.kind == kSchedPersistent && schedule == kSchedPersistent))
       return LQ_ERR_UNSUPPORTED_SHAPE;
-    if (s.kind == kSchedPersistent) s = make_schedule(M, N, K, lq::kPBT, kSchedTiles, 0, 0, dev->sms);
+    if (s.kind == kSchedPersistent)
+      s = make_schedule(M, N, K, lq::kPBT, kSchedTiles, 0, 0, dev->sms, dev->cluster_ctas);
   }
   st = check_schedule_shape(s, K);
   if (st != LQ_OK) return st;
@@ -601,8 +650,12 @@ size_t lq_w4a8_linear_workspace_size_ex(int M, int N, int K, int path) {
   if (path < LQ_LINEAR_AUTO || path > LQ_LINEAR_FUSED) return 0;
   DeviceInfo* dev = nullptr;
   int sms = 148;
-  if (current_device(&dev) == LQ_OK) sms = dev->sms;
-  const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, sms);
+  const int* cl = nullptr;
+  if (current_device(&dev) == LQ_OK) {
+    sms = dev->sms;
+    cl = dev->cluster_ctas;
+  }
+  const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, sms, cl);
   if (use_fused(s, M, path)) return 0;
   return align16((size_t)M * K) + align16((size_t)M * 4) + s.ws_bytes;
 }
@@ -633,7 +686,7 @@ lq_status lq_w4a8_linear_ex(const void* X_bf16, const uint8_t* qw, const uint8_t
   st = current_device(&dev);
   if (st != LQ_OK) return st;
   if (!device_addressable(X_bf16) || !device_addressable(out_bf16)) return LQ_ERR_INVALID_ARG;
-  const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, dev->sms);
+  const Schedule s = make_schedule(M, N, K, 0, 0, 0, 0, dev->sms, dev->cluster_ctas);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (path == LQ_LINEAR_FUSED && !fused_eligible(s, M)) return LQ_ERR_UNSUPPORTED_SHAPE;
   if (!use_fused(s, M, path)) {
@@ -737,8 +790,12 @@ size_t lq_w4a8_gemm_workspace_size_ex(int M, int N, int K, int block_t, int sche
   if (!valid_schedule(M, block_t, schedule, split_k, grid)) return 0;
   DeviceInfo* dev = nullptr;
   int sms = 148;
-  if (current_device(&dev) == LQ_OK) sms = dev->sms;
-  return make_schedule(M, N, K, block_t, schedule, split_k, grid, sms).ws_bytes;
+  const int* cl = nullptr;
+  if (current_device(&dev) == LQ_OK) {
+    sms = dev->sms;
+    cl = dev->cluster_ctas;
+  }
+  return make_schedule(M, N, K, block_t, schedule, split_k, grid, sms, cl).ws_bytes;
 }
 
 size_t lq_w4a8_gemm_workspace_size(int M, int N, int K) {
@@ -782,18 +839,35 @@ lq_status lq_w4a8_gemm_i32(const int8_t* x_q, const uint8_t* qw, const uint8_t* 
                    0, 0, 0, true, stream);
 }
 
-lq_status lq_plan_gemm(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms, int* plan) {
+lq_status lq_plan_gemm_ex(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms,
+                          const int* cluster_ctas, int* plan) {
   if (!plan || sms < 1) return LQ_ERR_INVALID_ARG;
+  if (cluster_ctas)
+    for (int i = 0; i < 3; ++i)
+      if (cluster_ctas[i] < 1) return LQ_ERR_INVALID_ARG;
   lq_status st = check_gemm_shape(M, N, K, LQ_GROUP);
   if (st != LQ_OK) return st;
   if (M < 1 || !valid_schedule(M, block_t, schedule, split_k, grid)) return LQ_ERR_INVALID_ARG;
-  const Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, sms);
+  const Schedule s = make_schedule(M, N, K, block_t, schedule, split_k, grid, sms, cluster_ctas);
   st = check_schedule_shape(s, K);
   if (st != LQ_OK) return st;
   plan[0] = s.kind;
   plan[1] = s.bt;
   plan[2] = s.cs;
   plan[3] = s.grid;
+  return LQ_OK;
+}
+
+lq_status lq_plan_gemm(int M, int N, int K, int block_t, int schedule, int split_k, int grid, int sms, int* plan) {
+  return lq_plan_gemm_ex(M, N, K, block_t, schedule, split_k, grid, sms, nullptr, plan);
+}
+
+lq_status lq_device_cluster_ctas(int* cluster_ctas) {
+  if (!cluster_ctas) return LQ_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  const lq_status st = current_device(&dev);
+  if (st != LQ_OK) return st;
+  for (int i = 0; i < 3; ++i) cluster_ctas[i] = dev->cluster_ctas[i];
   return LQ_OK;
 }
 
@@ -905,7 +979,7 @@ lq_status lq_w4a8_gemm_noalloc(const int8_t* x_q, const float* s_x, const uint8_
   DeviceInfo* dev = nullptr;
   st = current_device(&dev);
   if (st != LQ_OK) return st;
-  const Schedule s = make_schedule(M, N, K, 0, kSchedStreamK, 0, 0, dev->sms);
+  const Schedule s = make_schedule(M, N, K, 0, kSchedStreamK, 0, 0, dev->sms, dev->cluster_ctas);
   if (s.ws_bytes > kNoAllocScratchBytes) return LQ_ERR_WORKSPACE;
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
@@ -960,8 +1034,9 @@ lq_status grouped_impl(const int8_t* x_q, const float* s_x, const uint8_t* qw, c
   if (!device_addressable(out)) return LQ_ERR_INVALID_ARG;
   const long long tm_bound = std::min<long long>(((long long)M + (long long)groups * (bt - 1)) / bt, M);
   if (tm_bound * bt > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
-  const Schedule s = pair ? make_schedule((int)(tm_bound * bt), N, K, 0, kSchedPair, 0, 0, dev->sms)
-                          : make_schedule((int)(tm_bound * bt), N, K, bt, kSchedTiles, split_k, 0, dev->sms);
+  const Schedule s =
+      pair ? make_schedule((int)(tm_bound * bt), N, K, 0, kSchedPair, 0, 0, dev->sms, dev->cluster_ctas)
+           : make_schedule((int)(tm_bound * bt), N, K, bt, kSchedTiles, split_k, 0, dev->sms, dev->cluster_ctas);
   const int NT = groups * N;
   // the pair kernel loads 128 tokens and 128 weight rows per CTA with 256 K per stage
   const uint32_t x_rows = pair ? 128u : (uint32_t)bt;
@@ -1059,9 +1134,9 @@ lq_status launch_f8_bt(const Schedule& s, const CUtensorMap& tx, const void* x_f
 }
 
 lq_status w4f8_impl(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4, const float* s_w, void* out, int M,
-                    int N, int K, int sms, cudaStream_t st) {
+                    int N, int K, int sms, const int* cl, cudaStream_t st) {
   const int bt = M <= 16 ? 16 : M <= 64 ? 64 : 128;
-  const Schedule s = make_schedule(M, N, K, bt, kSchedTiles, 0, 0, sms);
+  const Schedule s = make_schedule(M, N, K, bt, kSchedTiles, 0, 0, sms, cl);
   if (s.tiles * s.cs > INT_MAX) return LQ_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap tx, tw;
   if (!make_map_u8(&tx, x_f8, (uint64_t)K, (uint64_t)M, (uint64_t)K, lq::kBlockK, (uint32_t)bt,
@@ -1141,7 +1216,8 @@ lq_status lq_w4f8_gemm(const uint8_t* x_f8, const float* s_x, const uint8_t* qw4
   st = current_device(&dev);
   if (st != LQ_OK) return st;
   if (!device_addressable(out_bf16)) return LQ_ERR_INVALID_ARG;
-  return w4f8_impl(x_f8, s_x, qw4, s_w, out_bf16, M, N, K, dev->sms, static_cast<cudaStream_t>(stream));
+  return w4f8_impl(x_f8, s_x, qw4, s_w, out_bf16, M, N, K, dev->sms, dev->cluster_ctas,
+                   static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
