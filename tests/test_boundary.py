@@ -3,6 +3,7 @@ include/lq.h, and rejects bad arguments before touching a device (no GPU needed)
 import ctypes
 
 import pytest
+import torch
 
 import w4a8_bit_weight_b200 as lq
 from w4a8_bit_weight_b200 import build as lqbuild
@@ -234,6 +235,19 @@ def test_plan_ex_rejects_bad_cluster_table(lib):
     assert _plan_ex(lib, 16, 4096, 4096, (296, 0, 264))[0] == 1
     assert _plan_ex(lib, 16, 4096, 4096, (296, 284, -1))[0] == 1
     assert lib.lq_device_cluster_ctas(None) == 1
+
+
+def test_cluster_table_never_exceeds_two_per_sm(lib):
+    # a table larger than two CTAs per SM counts as two per SM
+    for M, N, K in ((16, 4352, 14336), (16, 14336, 4096), (16, 4096, 4096)):
+        assert _plan_ex(lib, M, N, K, (10 ** 6,) * 3) == _plan_ex(lib, M, N, K, None)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the answer without a device")
+def test_device_cluster_table_needs_a_device(lib):
+    out = (ctypes.c_int * 3)(-7, -7, -7)
+    assert lib.lq_device_cluster_ctas(out) == 5  # LQ_ERR_CUDA
+    assert tuple(out) == (-7, -7, -7)
 
 
 def test_plan_follows_explicit_choices(lib):
